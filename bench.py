@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of the channel-wise gated delta-rule hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  gdelta_state_init (S <- 0)  ->  gdelta_fwd_chunked over the batch
+  (S_in = S_out = S)  ->  one gdelta_decode_step continuing every head.
+Workload (per GPU): B=4, T=4096, H=16, d_k=d_v=128, chunk 64, bf16 tokens,
+fp32 log-decay and state -- the Muir 1.34B-scale layer (the Muir review's
+d=2048 model: 16 heads of 128; 4096-token training length), synthetic data
+from ``synth``.  The inputs (680 MB) are larger than the 126 MB L2, so no L2
+flush is needed between steps.
+
+A second measurement times the decode step alone on batch 64 x 16 heads (fp32
+state of 67 MB, which fits in L2), flushing L2 between steps.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+N > 1 is launched with torchrun (one process per GPU); every rank runs its own
+batch (independent heads, no collective on the data path) and rank 0 prints
+one JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("gated-delta chunked fwd tokens/s (H=16,dk=dv=128); decode-step state HBM GB/s")
+WORKLOAD = "muir1b3_bf16"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- plumbing
+
+def dist_init(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, local, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+def fwd_bytes(B, T, H, dk, dv, tok_bytes):
+    """Algorithmic HBM bytes of one chunked-forward launch: q,k,z,b (d_k) and
+    v,w,g (d_v) tokens, fp32 log-decay, y, the fp32 state read and written."""
+    per_token_head = 4 * dk * tok_bytes + 3 * dv * tok_bytes + 4 * dk + dv * tok_bytes
+    return B * T * H * per_token_head + 2 * B * H * dk * dv * 4 + H * dk * 4
+
+
+def decode_bytes(B, H, dk, dv, tok_bytes):
+    """Algorithmic bytes of one decode step: state read + write, the token
+    vectors, the fp32 log-decay and y."""
+    return B * H * (2 * dk * dv * 4 + 4 * dk * tok_bytes + 3 * dv * tok_bytes + 4 * dk
+                    + dv * tok_bytes) + H * dk * 4
+
+
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str):
+    """Per-launch DRAM bytes recorded from an ncu capture of the current
+    source of ``kernel_file`` (profiles/traffic.json), else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel_file)
+        if rec and rec.get("source_sha") == source_digest([kernel_file]):
+            return float(rec["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, local, world):
+    import channel_gated_delta_b200 as gd
+    import synth
+
+    dev = torch.device("cuda", local)
+    shape = synth.CONFIGS[WORKLOAD]
+    B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+    host = synth.generate(shape, seed=shape.seed + 1000 * rank)
+    d = {k: v.to(dev) for k, v in host.items()}
+    S = torch.empty(B, H, dk, dv, device=dev)
+    y = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    step_tok = synth.decode_step_inputs(0, seed=77 + rank, B=B, H=H, dk=dk, dv=dv)
+    dtok = {k: v.to(dev) for k, v in step_tok.items()}
+    y_dec = torch.empty(B, H, dv, dtype=torch.bfloat16, device=dev)
+    path = gd.gdelta_fwd_selected_path(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                       d["log_alpha"], chunk=C, path=args.path)
+    ws_bytes = gd.gdelta_fwd_workspace_bytes(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                             d["log_alpha"], chunk=C, path=args.path)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        gd.gdelta_state_init(S, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"],
+                              gamma_stat=d["gamma_stat"], S_in=S, S_out=S, y=y, chunk=C,
+                              path=args.path, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        gd.gdelta_decode_step(dtok["q"], dtok["k"], dtok["v"], dtok["b"], dtok["w"], dtok["z"],
+                              dtok["g"], dtok["log_alpha"], S, gamma_stat=d["gamma_stat"], y=y_dec,
+                              stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if gd.gdelta_get_last_device_error(stream) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    clocks = ClockSampler(dev.index if world == 1 else local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    fwd_avg_ms = max_over_ranks(sum(fwd_ms) / len(fwd_ms), world)
+
+    tok_per_step = B * T + B                       # prefill tokens + one decode token per row
+    value = tok_per_step * world / (ms_step * 1e-3)
+    hbm, peak_kind = peaks()
+    fb = fwd_bytes(B, T, H, dk, dv, 2)
+    achieved = fb / (fwd_avg_ms * 1e-3) / 1e9
+    kernel_file = ("channel_gated_delta_b200/csrc/fwd_tc.cu" if path == "tc"
+                   else "channel_gated_delta_b200/csrc/fwd_simt.cu")
+    traffic = recorded_traffic(kernel_file)
+
+    # ---- decode-only measurement (batch 64 x 16 heads, L2 flushed between steps)
+    dec = run_decode(args, dev, stream, rank, world) if args.decode_steps > 0 else None
+
+    # ---- end to end through the public API with host buffers
+    e2e = None if args.no_e2e else run_e2e(args, gd, host, dev, stream, shape, world, path)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(host, shape)
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32" if path == "simt" else "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{WORKLOAD}: B{B} T{T} H{H} dk=dv={dk} chunk {C}, bf16 tokens, fp32 log-decay and state",
+            "step": "state_init + fwd_chunked + 1 decode step (all heads)",
+            "tokens_per_step_per_gpu": tok_per_step,
+            "kernel_path": path,
+            "workspace_bytes": ws_bytes,
+            "l2": "inputs (680 MB per GPU) larger than the 126 MB L2; no flush",
+            "parallelism": f"dp{world} (independent batches per GPU, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "gdn2_fwd_tc_kernel" if path == "tc" else "gdn2_fwd_simt_kernel",
+            "achieved": achieved,
+            "peak": hbm,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "unit": "GB/s",
+            "frac": achieved / hbm,
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": fb,
+            "launch_ms": fwd_avg_ms,
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "decode": dec,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, dev, stream, rank, world):
+    import channel_gated_delta_b200 as gd
+    import synth
+    D = synth.DECODE
+    B, H, dk, dv = D["B"], D["H"], D["dk"], D["dv"]
+    gen = torch.Generator(device="cpu").manual_seed(5 + rank)
+    S = (torch.randn(B, H, dk, dv, generator=gen) * 0.05).to(dev)
+    gamma = synth.decode_gamma().to(dev)
+    pool = [{k: v.to(dev) for k, v in synth.decode_step_inputs(i, B=B, H=H, dk=dk, dv=dv).items()}
+            for i in range(8)]
+    y = torch.empty(B, H, dv, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def one(i):
+        t = pool[i % len(pool)]
+        gd.gdelta_decode_step(t["q"], t["k"], t["v"], t["b"], t["w"], t["z"], t["g"], t["log_alpha"],
+                              S, gamma_stat=gamma, y=y, stream=stream)
+
+    for i in range(5):
+        one(i)
+    n = args.decode_steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier(world)
+    for i in range(n):
+        flush.zero_()                                   # evict the state from L2 (untimed)
+        evs[i][0].record(stream)
+        one(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    med = max_over_ranks(statistics.median(ms), world)
+    mean = max_over_ranks(sum(ms) / n, world)
+    nb = decode_bytes(B, H, dk, dv, 2)
+    hbm, kind = peaks()
+    gbs = nb / (med * 1e-3) / 1e9
+    return {
+        "workload": f"decode B{B} H{H} dk=dv={dk}, fp32 state {B * H * dk * dv * 4 / 1e6:.1f} MB, bf16 tokens",
+        "value": gbs * world,
+        "unit": "GB/s",
+        "per_gpu_gbs": gbs,
+        "steps_per_s": 1e3 / med,
+        "tokens_per_s": B * world * 1e3 / med,
+        "ms_per_step_median": med,
+        "ms_per_step_mean": mean,
+        "timed_steps": n,
+        "bytes_per_step": nb,
+        "roofline": {"bound": "hbm", "kernel": "gdn2_decode_kernel", "achieved": gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": gbs / hbm,
+                     "traffic": recorded_traffic("channel_gated_delta_b200/csrc/decode.cu")},
+        "l2": "256 MB buffer written between timed steps (state evicted)",
+        "state_init": "random N(0, 0.05^2) state (timing does not depend on values)",
+    }
+
+
+def run_e2e(args, gd, host, dev, stream, shape, world, path):
+    """Same step through the public API, inputs copied from pinned host memory
+    every step and y / S read back, all inside the timed region."""
+    B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+    keys = ("q", "k", "v", "b", "w", "z", "g", "log_alpha", "gamma_stat")
+    hp = {k: host[k].pin_memory() for k in keys}
+    dd = {k: torch.empty_like(host[k], device=dev) for k in keys}
+    S = torch.empty(B, H, dk, dv, device=dev)
+    y = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    y_h = torch.empty(B, T, H, dv, dtype=torch.bfloat16).pin_memory()
+    S_h = torch.empty(B, H, dk, dv).pin_memory()
+    ws_bytes = gd.gdelta_fwd_workspace_bytes(dd["q"], dd["k"], dd["v"], dd["b"], dd["w"], dd["z"],
+                                             dd["g"], dd["log_alpha"], chunk=C, path=args.path)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    h2d = sum(hp[k].numel() * hp[k].element_size() for k in keys)
+    d2h = y_h.numel() * 2 + S_h.numel() * 4
+
+    def step():
+        with torch.cuda.stream(stream):
+            for k in keys:
+                dd[k].copy_(hp[k], non_blocking=True)
+        gd.gdelta_state_init(S, stream=stream)
+        gd.gdelta_fwd_chunked(dd["q"], dd["k"], dd["v"], dd["b"], dd["w"], dd["z"], dd["g"],
+                              dd["log_alpha"], gamma_stat=dd["gamma_stat"], S_in=S, S_out=S, y=y,
+                              chunk=C, path=args.path, workspace=ws, stream=stream)
+        with torch.cuda.stream(stream):
+            y_h.copy_(y, non_blocking=True)
+            S_h.copy_(S, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 5))
+    barrier(world)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b) / n, world)
+    return {"value": B * T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "api": "channel_gated_delta_b200.gdelta_state_init + gdelta_fwd_chunked (pinned host copies)"}
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def cpu_baseline(host, shape, heads=None):
+    """The float64 oracle as it stands, on this host's cores."""
+    import oracle
+    H, T = shape.H, shape.T
+    heads = heads if heads is not None else [(b, h) for b in range(shape.B) for h in range(H)]
+    sub = {k: v for k, v in host.items()}
+    t0 = time.perf_counter()
+    r = oracle.forward(sub, heads=heads)
+    dt = time.perf_counter() - t0
+    token_heads = len(heads) * T
+    return {"value": token_heads / H / dt, "unit": "tokens/s", "cores": r["threads"], "kind": "oracle",
+            "sample": f"{len(heads)} of {shape.B * H} heads x {T} tokens of the same workload "
+                      f"({token_heads} token-heads; tokens/s = token-heads/s / H), float64 C recurrence",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import synth
+    shape = synth.CONFIGS[WORKLOAD]
+    host = synth.generate(shape)
+    heads = [(0, h) for h in range(4)]
+    T = 1024
+    sub = {k: (v[:, :T] if v.dim() == 4 else v) for k, v in host.items()}
+    import oracle
+    for _ in range(args.warmup):
+        oracle.forward(sub, heads=heads)
+    t0 = time.perf_counter()
+    threads = 0
+    for _ in range(args.steps):
+        threads = oracle.forward(sub, heads=heads)["threads"]
+    dt = (time.perf_counter() - t0) / args.steps
+    value = len(heads) * T / shape.H / dt
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: B4 T4096 H16 dk=dv=128 chunk 64 (bounded sample per step)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {len(heads)} heads x {T} tokens of the workload, "
+                                   "float64 C recurrence on the host cores"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, local, world = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            if not torch.cuda.is_available():
+                raise RuntimeError("bench.py --impl ours needs a CUDA device")
+            run_ours(args, rank, local, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,212 @@
+"""B200 (sm_100a) channel-wise gated delta-rule token mixer.
+
+Thin Python binding over the C ABI in ``include/gdelta.h`` (library
+``libgdelta.so`` built in-tree by ``channel_gated_delta_b200.build``).  The
+functions carry the C names and do argument marshalling only; PyTorch supplies
+device memory and streams.  Every step of the mixer runs in the library's CUDA
+kernels and a missing library raises -- there is no CPU fallback.
+
+The operation (Muir review §2.1, GDN-2 update with the Muir readout), per head
+and token, row-vector convention::
+
+    S_hat = Diag(exp(log_alpha_t)) S
+    S     = S_hat - (b_t*k_t)^T (k_t S_hat) + k_t^T (w_t*v_t)
+    o_t   = (q_t * gamma_stat * 2 sigmoid(z_t)) S
+    y_t   = g_t * o_t / sqrt(mean(o_t^2) + eps)
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _native
+
+__all__ = [
+    "GdeltaError",
+    "gdelta_abi_version",
+    "gdelta_status_string",
+    "gdelta_fwd_workspace_bytes",
+    "gdelta_fwd_selected_path",
+    "gdelta_state_init",
+    "gdelta_fwd_chunked",
+    "gdelta_decode_step",
+    "gdelta_get_last_device_error",
+]
+
+
+class GdeltaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _native.STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{where}: {name} ({gdelta_status_string(status)})")
+
+
+def _lib():
+    return _native.load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != _native.GDELTA_OK:
+        raise GdeltaError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev_ptr(t: Optional[torch.Tensor], name: str, dtype=None, shape=None, required=True):
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _native.GDELTA_BF16
+    if t.dtype == torch.float32:
+        return _native.GDELTA_F32
+    raise ValueError(f"token tensors must be bf16 or fp32, got {t.dtype}")
+
+
+def gdelta_abi_version() -> int:
+    return int(_lib().gdelta_abi_version())
+
+
+def gdelta_status_string(status: int) -> str:
+    return _lib().gdelta_status_string(int(status)).decode()
+
+
+def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
+                path, workspace) -> _native.FwdArgs:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    a = _native.FwdArgs()
+    a.B, a.T, a.H, a.dk, a.dv = int(B), int(T), int(H), int(dk), int(dv)
+    a.chunk = int(chunk)
+    a.dtype = _dtype_code(q)
+    a.path = _native.PATHS[path]
+    ks, vs = (B, T, H, dk), (B, T, H, dv)
+    a.q = _dev_ptr(q, "q", dt, ks)
+    a.k = _dev_ptr(k, "k", dt, ks)
+    a.z = _dev_ptr(z, "z", dt, ks)
+    a.b = _dev_ptr(b, "b", dt, ks)
+    a.v = _dev_ptr(v, "v", dt, vs)
+    a.w = _dev_ptr(w, "w", dt, vs)
+    a.g = _dev_ptr(g, "g", dt, vs)
+    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, ks)
+    a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
+    a.S_in = _dev_ptr(S_in, "S_in", torch.float32, (B, H, dk, dv), required=False)
+    a.S_out = _dev_ptr(S_out, "S_out", torch.float32, (B, H, dk, dv), required=False)
+    a.y = _dev_ptr(y, "y", dt, vs, required=False)
+    a.o_raw = _dev_ptr(o_raw, "o_raw", torch.float32, vs, required=False)
+    a.eps = float(eps)
+    if workspace is not None:
+        a.workspace = _dev_ptr(workspace, "workspace")
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    return a
+
+
+def gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
+                               path: str = "auto") -> int:
+    a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
+                    path, None)
+    return int(_lib().gdelta_fwd_workspace_bytes(ctypes.byref(a)))
+
+
+def gdelta_fwd_selected_path(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
+                             path: str = "auto") -> str:
+    a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
+                    path, None)
+    code = int(_lib().gdelta_fwd_selected_path(ctypes.byref(a)))
+    if code < 0:
+        raise GdeltaError(2, "gdelta_fwd_selected_path")
+    return _native.PATH_NAMES[code]
+
+
+def gdelta_state_init(S: torch.Tensor, S_src: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """S <- 0 (S_src None) or S <- S_src.  S: [B,H,dk,dv] fp32 on the GPU."""
+    if S.dim() != 4:
+        raise ValueError("S must be [B, H, dk, dv]")
+    B, H, dk, dv = S.shape
+    p = _dev_ptr(S, "S", torch.float32)
+    ps = _dev_ptr(S_src, "S_src", torch.float32, tuple(S.shape), required=False)
+    _check(_lib().gdelta_state_init(p, B, H, dk, dv, ps, _stream(stream)), "gdelta_state_init")
+    return S
+
+
+def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=None, S_out=None,
+                       y=None, o_raw=None, chunk: int = 64, eps: float = 1e-6, path: str = "auto",
+                       workspace=None, return_state: bool = True, stream=None
+                       ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked forward over [B,T,H,d] tokens.  Returns (y, S_out).
+
+    Outputs not passed in are allocated with torch on q's device; S_out is
+    only allocated when ``return_state``.  ``workspace`` (uint8 CUDA tensor) is
+    allocated when the selected kernel needs one and none is given.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_out is None and return_state:
+        S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, chunk=chunk, path=path)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
+                    path, workspace)
+    _check(_lib().gdelta_fwd_chunked(ctypes.byref(a), _stream(stream)), "gdelta_fwd_chunked")
+    return y, S_out
+
+
+def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=None, o_raw=None,
+                       eps: float = 1e-6, stream=None) -> torch.Tensor:
+    """One token per (batch, head): S [B,H,dk,dv] fp32 updated in place; returns y [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if y is None:
+        y = torch.empty((B, H, dv), dtype=dt, device=q.device)
+    a = _native.DecodeArgs()
+    a.B, a.H, a.dk, a.dv = int(B), int(H), int(dk), int(dv)
+    a.dtype = _dtype_code(q)
+    a.reserved = 0
+    ks, vs = (B, H, dk), (B, H, dv)
+    a.q = _dev_ptr(q, "q", dt, ks)
+    a.k = _dev_ptr(k, "k", dt, ks)
+    a.z = _dev_ptr(z, "z", dt, ks)
+    a.b = _dev_ptr(b, "b", dt, ks)
+    a.v = _dev_ptr(v, "v", dt, vs)
+    a.w = _dev_ptr(w, "w", dt, vs)
+    a.g = _dev_ptr(g, "g", dt, vs)
+    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, ks)
+    a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
+    a.S = _dev_ptr(S, "S", torch.float32, (B, H, dk, dv))
+    a.y = _dev_ptr(y, "y", dt, vs)
+    a.o_raw = _dev_ptr(o_raw, "o_raw", torch.float32, vs, required=False)
+    a.eps = float(eps)
+    _check(_lib().gdelta_decode_step(ctypes.byref(a), _stream(stream)), "gdelta_decode_step")
+    return y
+
+
+def gdelta_get_last_device_error(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status code."""
+    return int(_lib().gdelta_get_last_device_error(_stream(stream)))

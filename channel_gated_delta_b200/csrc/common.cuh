@@ -1,0 +1,62 @@
+// Shared device helpers for the gated delta-rule kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdelta.h"
+
+namespace gdelta {
+
+// Element loads/stores for the two token dtypes.
+__device__ __forceinline__ float ldf(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void stf(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// 2 * sigmoid(z): the dynamic readout modulation in (0, 2) (Muir review §2.1).
+__device__ __forceinline__ float two_sigmoid(float z) { return 2.0f / (1.0f + expf(-z)); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Device status codes written by kernels that detect a run-time fault.
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1 };
+
+struct FwdParams {
+    int B, T, H, dk, dv, C;
+    const void *q, *k, *z, *b, *v, *w, *g;
+    const float *la, *gs, *S_in;
+    float *S_out;
+    void *y;
+    float *o_raw;
+    float eps;
+    int *status;
+};
+
+struct DecodeParams {
+    int B, H, dk, dv;
+    const void *q, *k, *z, *b, *v, *w, *g;
+    const float *la, *gs;
+    float *S;
+    void *y;
+    float *o_raw;
+    float eps;
+};
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t stream);
+cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
+size_t fwd_simt_smem_bytes(int dk, int dv, int C);
+int fwd_simt_chunk(int dk, int dv, int requested);
+cudaError_t launch_state_init(float *S, const float *src, size_t n, cudaStream_t stream);
+
+}  // namespace gdelta

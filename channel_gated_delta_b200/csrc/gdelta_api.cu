@@ -1,0 +1,161 @@
+// C ABI entry points: argument checks on the host, then kernel launches on the
+// caller's stream.  Nothing here allocates device memory.
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace gdelta {
+
+// Device status word (one per device that loads the library).  Kernels that
+// detect a run-time fault (a bounded wait that ran out) write a nonzero code.
+__device__ int g_device_status;
+
+static int *status_ptr() {
+    static std::mutex mu;
+    static int *ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = (int *)p;
+    }
+    return ptrs[dev];
+}
+
+static bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+static bool dim_ok(int d) { return d == 64 || d == 128; }
+
+static gdelta_status check_fwd(const gdelta_fwd_args *a) {
+    if (!a) return GDELTA_ERR_INVALID_ARG;
+    if (a->B < 1 || a->H < 1 || a->T < 0) return GDELTA_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return GDELTA_ERR_INVALID_ARG;
+    if (a->dtype != GDELTA_F32 && a->dtype != GDELTA_BF16) return GDELTA_ERR_UNSUPPORTED;
+    if (!dim_ok(a->dk) || !dim_ok(a->dv)) return GDELTA_ERR_UNSUPPORTED;
+    const int C = a->chunk == 0 ? 64 : a->chunk;
+    if (C != 16 && C != 32 && C != 64) return GDELTA_ERR_UNSUPPORTED;
+    if (a->path < GDELTA_PATH_AUTO || a->path > GDELTA_PATH_TC) return GDELTA_ERR_INVALID_ARG;
+    if (a->T > 0) {
+        if (!a->q || !a->k || !a->z || !a->b || !a->v || !a->w || !a->g || !a->log_alpha || !a->y)
+            return GDELTA_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->gamma_stat,
+                          a->S_in, a->S_out, a->y, a->o_raw, a->workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
+    return GDELTA_OK;
+}
+
+static int select_path(const gdelta_fwd_args *a) {
+    // The tensor-core kernel is not part of this build yet: every shape runs
+    // on the fp32 CUDA-core kernel.
+    if (a->path == GDELTA_PATH_TC) return -1;
+    return GDELTA_PATH_SIMT;
+}
+
+}  // namespace gdelta
+
+using namespace gdelta;
+
+extern "C" {
+
+int gdelta_abi_version(void) { return GDELTA_ABI_VERSION; }
+
+const char *gdelta_status_string(gdelta_status s) {
+    switch (s) {
+        case GDELTA_OK: return "ok";
+        case GDELTA_ERR_INVALID_ARG: return "invalid argument";
+        case GDELTA_ERR_UNSUPPORTED: return "unsupported shape, chunk, dtype or path";
+        case GDELTA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case GDELTA_ERR_CUDA: return "CUDA error";
+        case GDELTA_ERR_TIMEOUT: return "device-side bounded wait ran out";
+        case GDELTA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int gdelta_fwd_selected_path(const gdelta_fwd_args *args) {
+    if (check_fwd(args) != GDELTA_OK) return -1;
+    return select_path(args);
+}
+
+size_t gdelta_fwd_workspace_bytes(const gdelta_fwd_args *args) {
+    if (check_fwd(args) != GDELTA_OK) return 0;
+    return 0;
+}
+
+gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32_t dk, int32_t dv,
+                                const float *S_src, void *stream) {
+    if (!S || B < 1 || H < 1) return GDELTA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDELTA_ERR_UNSUPPORTED;
+    if (!aligned16(S) || !aligned16(S_src)) return GDELTA_ERR_ALIGNMENT;
+    const size_t n = (size_t)B * H * dk * dv;
+    if (S_src && S_src != S) {
+        const char *a = (const char *)S, *b = (const char *)S_src;
+        if (a < b + n * sizeof(float) && b < a + n * sizeof(float)) return GDELTA_ERR_INVALID_ARG;
+    }
+    return launch_state_init(S, S_src, n, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
+                                                                               : GDELTA_ERR_CUDA;
+}
+
+gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
+    gdelta_status st = check_fwd(a);
+    if (st != GDELTA_OK) return st;
+    const int path = select_path(a);
+    if (path < 0) return GDELTA_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (a->T == 0) {
+        if (!a->S_out) return GDELTA_OK;
+        return launch_state_init(a->S_out, a->S_in, (size_t)a->B * a->H * a->dk * a->dv, s) ==
+                       cudaSuccess
+                   ? GDELTA_OK
+                   : GDELTA_ERR_CUDA;
+    }
+    FwdParams p;
+    p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv;
+    p.q = a->q; p.k = a->k; p.z = a->z; p.b = a->b; p.v = a->v; p.w = a->w; p.g = a->g;
+    p.la = a->log_alpha; p.gs = a->gamma_stat; p.S_in = a->S_in; p.S_out = a->S_out;
+    p.y = a->y; p.o_raw = a->o_raw; p.eps = a->eps;
+    p.status = status_ptr();
+    p.C = fwd_simt_chunk(a->dk, a->dv, a->chunk == 0 ? 64 : a->chunk);
+    if (p.C == 0) return GDELTA_ERR_UNSUPPORTED;
+    return launch_fwd_simt(p, a->dtype, s) == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
+}
+
+gdelta_status gdelta_decode_step(const gdelta_decode_args *a, void *stream) {
+    if (!a) return GDELTA_ERR_INVALID_ARG;
+    if (a->B < 1 || a->H < 1 || a->reserved != 0) return GDELTA_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return GDELTA_ERR_INVALID_ARG;
+    if (a->dtype != GDELTA_F32 && a->dtype != GDELTA_BF16) return GDELTA_ERR_UNSUPPORTED;
+    if (!dim_ok(a->dk) || !dim_ok(a->dv)) return GDELTA_ERR_UNSUPPORTED;
+    if (!a->q || !a->k || !a->z || !a->b || !a->v || !a->w || !a->g || !a->log_alpha || !a->S || !a->y)
+        return GDELTA_ERR_INVALID_ARG;
+    const void *ptrs[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->gamma_stat,
+                          a->S, a->y, a->o_raw};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
+    DecodeParams p;
+    p.B = a->B; p.H = a->H; p.dk = a->dk; p.dv = a->dv;
+    p.q = a->q; p.k = a->k; p.z = a->z; p.b = a->b; p.v = a->v; p.w = a->w; p.g = a->g;
+    p.la = a->log_alpha; p.gs = a->gamma_stat; p.S = a->S; p.y = a->y; p.o_raw = a->o_raw;
+    p.eps = a->eps;
+    return launch_decode(p, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
+                                                                           : GDELTA_ERR_CUDA;
+}
+
+gdelta_status gdelta_get_last_device_error(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDELTA_ERR_CUDA;
+    int *p = status_ptr();
+    if (!p) return GDELTA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GDELTA_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    }
+    return v == kDevOk ? GDELTA_OK : GDELTA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

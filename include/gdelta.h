@@ -1,0 +1,186 @@
+/*
+ * gdelta.h -- C ABI of the channel-wise gated delta-rule token mixer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The mixer (GDN-2 state update with the Muir readout).  Per head it keeps a
+ * fixed d_k x d_v fp32 state S.  For every token t (row-vector convention,
+ * k_t, q_t in R^{1 x d_k}, v_t in R^{1 x d_v}):
+ *
+ *   S_hat = Diag(alpha_t) S_{t-1},            alpha_t = exp(log_alpha_t)
+ *   S_t   = S_hat - (b_t*k_t)^T (k_t S_hat) + k_t^T (w_t*v_t)
+ *   o_t   = (q_t * gamma_stat * 2 sigmoid(z_t)) S_t
+ *   y_t   = g_t * o_t / sqrt(mean_j o_tj^2 + eps)
+ *
+ * Sources: "Muir: Linear Attention with Sensitivity-Allocated Gating and
+ * Matched-Filter Readout" (arXiv:2611.08376), review page §2.1 (per-channel
+ * decay alpha in (0,1)^{d_k}, erase gate b in (0,2)^{d_k} on the key, write
+ * gate w in (0,1)^{d_v} on the value, query-only readout gain, per-head RMSNorm
+ * followed by the output gate) and §2.4 (chunked kernel); "Kimi3 = GPT2 x
+ * 22580" §3-§4 (the state is the cache; read after write; chunked prefill).
+ * The page elides the update's display equation; the form above is the one
+ * whose special cases are KDA (b = w = beta), Gated DeltaNet (scalar alpha)
+ * and DeltaNet (alpha = 1), as the ETH DeltaNet-family study states in its
+ * "Gated DeltaNet-2" section.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    owned by the caller.  The library allocates no device memory and keeps
+ *    no state between calls except cached kernel attributes.
+ *  - Token tensors are contiguous [B, T, H, d] (d innermost); decode tensors
+ *    are [B, H, d]; states are [B, H, d_k, d_v] fp32 (d_v innermost).
+ *  - Every pointer must be 16-byte aligned (GDELTA_ERR_ALIGNMENT otherwise).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  They return after the launches are queued.
+ *  - Errors are return codes; nothing aborts or throws across the ABI.
+ *    Argument checks run on the host before any launch.  A launch failure is
+ *    GDELTA_ERR_CUDA.  Kernels that detect a fault at run time (a bounded wait
+ *    that ran out) record it in a device status word that
+ *    gdelta_get_last_device_error() reads.
+ */
+#ifndef GDELTA_H
+#define GDELTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDELTA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDELTA_API __attribute__((visibility("default")))
+#else
+#define GDELTA_API
+#endif
+
+typedef enum gdelta_status {
+    GDELTA_OK = 0,
+    GDELTA_ERR_INVALID_ARG = 1,   /* null pointer where one is required, bad size */
+    GDELTA_ERR_UNSUPPORTED = 2,   /* shape / chunk / dtype outside the supported set */
+    GDELTA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    GDELTA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    GDELTA_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (device status) */
+    GDELTA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} gdelta_status;
+
+typedef enum gdelta_dtype {
+    GDELTA_F32 = 0,               /* q,k,v,b,w,z,g and y are fp32 */
+    GDELTA_BF16 = 1               /* q,k,v,b,w,z,g and y are bf16 */
+} gdelta_dtype;
+
+/* Kernel selection for gdelta_fwd_chunked (args.path). */
+typedef enum gdelta_fwd_path {
+    GDELTA_PATH_AUTO = 0,         /* tensor-core path where supported, else SIMT */
+    GDELTA_PATH_SIMT = 1,         /* fp32 CUDA-core chunked kernel (any supported shape) */
+    GDELTA_PATH_TC = 2            /* tcgen05 tensor-core chunked kernel (bf16, d = 128, C = 64) */
+} gdelta_fwd_path;
+
+/*
+ * Chunked forward (prefill / training forward) over T tokens.
+ *
+ *   q, k, z, b : [B, T, H, d_k]  dtype        query, key, readout logit, erase gate
+ *   v, w, g    : [B, T, H, d_v]  dtype        value, write gate, output gate
+ *   log_alpha  : [B, T, H, d_k]  fp32, <= 0   log of the per-channel decay
+ *   gamma_stat : [H, d_k]        fp32         static readout profile; NULL = ones
+ *   S_in       : [B, H, d_k, d_v] fp32        state before token 0; NULL = zeros
+ *   S_out      : [B, H, d_k, d_v] fp32        state after token T-1; NULL = not
+ *                                             written; may equal S_in (in place)
+ *   y          : [B, T, H, d_v]  dtype        gated, normalised readout
+ *   o_raw      : [B, T, H, d_v]  fp32         optional pre-norm readout o_t; NULL
+ *                                             = not written
+ *   chunk      : tokens per chunk; 0 = 64.  Results do not depend on it beyond
+ *                rounding.  A ragged last chunk (T % chunk != 0) is handled
+ *                inside the kernels.
+ *   eps        : RMSNorm epsilon (the workloads use 1e-6).
+ *   path       : gdelta_fwd_path.
+ *   workspace  : device scratch of gdelta_fwd_workspace_bytes(args) bytes
+ *                (may be NULL when that is 0).
+ *
+ * Supported: d_k, d_v in {64, 128}; chunk in {16, 32, 64}; B, H >= 1; T >= 0
+ * (T = 0 only copies S_in to S_out).
+ */
+typedef struct gdelta_fwd_args {
+    int32_t B, T, H, dk, dv;
+    int32_t chunk;
+    int32_t dtype;        /* gdelta_dtype */
+    int32_t path;         /* gdelta_fwd_path */
+    const void *q, *k, *z, *b;
+    const void *v, *w, *g;
+    const float *log_alpha;
+    const float *gamma_stat;
+    const float *S_in;
+    float *S_out;
+    void *y;
+    float *o_raw;
+    float eps;
+    void *workspace;
+    size_t workspace_bytes;
+} gdelta_fwd_args;
+
+/*
+ * One decode step for B x H heads (one token each), updating S in place.
+ * Same operation as one token of the chunked forward ("Kimi3 = GPT2 x 22580"
+ * §1/§3: decoding reads and rewrites the fixed-size cache).
+ *
+ *   q, k, z, b : [B, H, d_k] dtype;  v, w, g : [B, H, d_v] dtype
+ *   log_alpha  : [B, H, d_k] fp32;   gamma_stat : [H, d_k] fp32 or NULL
+ *   S          : [B, H, d_k, d_v] fp32, read as S_{t-1}, overwritten with S_t
+ *   y          : [B, H, d_v] dtype;  o_raw : [B, H, d_v] fp32 or NULL
+ */
+typedef struct gdelta_decode_args {
+    int32_t B, H, dk, dv;
+    int32_t dtype;        /* gdelta_dtype */
+    int32_t reserved;     /* must be 0 */
+    const void *q, *k, *z, *b;
+    const void *v, *w, *g;
+    const float *log_alpha;
+    const float *gamma_stat;
+    float *S;
+    void *y;
+    float *o_raw;
+    float eps;
+} gdelta_decode_args;
+
+/* ABI version of the loaded library (GDELTA_ABI_VERSION it was built with). */
+GDELTA_API int gdelta_abi_version(void);
+
+/* Static, never-NULL description of a status code. */
+GDELTA_API const char *gdelta_status_string(gdelta_status status);
+
+/* Bytes of device workspace gdelta_fwd_chunked needs for these arguments
+ * (0 when the selected kernel needs none).  Returns 0 for invalid arguments;
+ * gdelta_fwd_chunked reports those. */
+GDELTA_API size_t gdelta_fwd_workspace_bytes(const gdelta_fwd_args *args);
+
+/* Which kernel gdelta_fwd_chunked would run for these arguments
+ * (GDELTA_PATH_SIMT or GDELTA_PATH_TC), or -1 if the arguments are invalid. */
+GDELTA_API int gdelta_fwd_selected_path(const gdelta_fwd_args *args);
+
+/*
+ * State initialisation ("Kimi3 = GPT2 x 22580" §3: S starts at zero, or at
+ * the cache a previous call returned).  S[B,H,d_k,d_v] fp32 <- 0 when S_src is
+ * NULL, else <- S_src (same shape; must not overlap S unless equal).
+ */
+GDELTA_API gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32_t dk, int32_t dv,
+                                const float *S_src, void *stream);
+
+/* Chunked forward; see gdelta_fwd_args. */
+GDELTA_API gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *args, void *stream);
+
+/* One decode step; see gdelta_decode_args. */
+GDELTA_API gdelta_status gdelta_decode_step(const gdelta_decode_args *args, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns GDELTA_OK, GDELTA_ERR_TIMEOUT (a kernel's bounded
+ * wait ran out) or GDELTA_ERR_CUDA (the synchronisation itself failed).
+ */
+GDELTA_API gdelta_status gdelta_get_last_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDELTA_H */

@@ -1,0 +1,86 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from channel_gated_delta_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdelta.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDELTA_API\s+[\w\s\*]*?\b(gdelta_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_native.LIB_PATH):
+        from channel_gated_delta_b200 import build
+        build.build()
+    return _native.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_native.EXPORTED)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.gdelta_abi_version() == 1
+    for code in range(7):
+        s = lib.gdelta_status_string(code)
+        assert s and s != b"unknown status"
+    assert lib.gdelta_status_string(99) == b"unknown status"
+
+
+def _args(**kw):
+    a = _native.FwdArgs()
+    a.B, a.T, a.H, a.dk, a.dv, a.chunk, a.dtype, a.path = 1, 64, 1, 128, 128, 64, 1, 0
+    fake = 0x10000
+    for i, n in enumerate(("q", "k", "z", "b", "v", "w", "g", "log_alpha", "y")):
+        setattr(a, n, fake + 256 * i)
+    a.eps = 1e-6
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def test_host_validation_codes(lib):
+    f = lib.gdelta_fwd_chunked
+    assert f(None, None) == 1
+    assert f(ctypes.byref(_args(B=0)), None) == 1
+    assert f(ctypes.byref(_args(T=-1)), None) == 1
+    assert f(ctypes.byref(_args(dk=96)), None) == 2
+    assert f(ctypes.byref(_args(chunk=48)), None) == 2
+    assert f(ctypes.byref(_args(dtype=7)), None) == 2
+    assert f(ctypes.byref(_args(path=9)), None) == 1
+    assert f(ctypes.byref(_args(q=None)), None) == 1
+    assert f(ctypes.byref(_args(k=0x10001)), None) == 3
+    assert f(ctypes.byref(_args(eps=float("nan"))), None) == 1
+    assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(B=0))) == -1
+    assert lib.gdelta_fwd_workspace_bytes(ctypes.byref(_args(B=0))) == 0
+    assert lib.gdelta_state_init(None, 1, 1, 128, 128, None, None) == 1
+    assert lib.gdelta_state_init(0x10000, 1, 1, 100, 128, None, None) == 2
+    assert lib.gdelta_state_init(0x10004, 1, 1, 128, 128, None, None) == 3
+    # overlapping, unequal source and destination
+    assert lib.gdelta_state_init(0x10000, 1, 1, 128, 128, 0x10010, None) == 1
+    d = _native.DecodeArgs()
+    d.B, d.H, d.dk, d.dv, d.dtype, d.reserved = 1, 1, 128, 128, 1, 0
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # null tensors
+    d.reserved = 3
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
+
+
+def test_path_selection_is_host_logic(lib):
+    a = _args()
+    assert lib.gdelta_fwd_selected_path(ctypes.byref(a)) in (1, 2)
+    assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(dtype=0))) == 1
+    assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(path=1))) == 1

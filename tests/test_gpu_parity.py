@@ -1,0 +1,202 @@
+"""GPU path vs the float64 oracle, element by element on the same seeded
+inputs, through the C ABI.  Tolerances are max|diff| / rms(reference):
+1e-4 for fp32 inputs, 2e-2 for bf16 inputs / fp32 accumulation."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_util import TOL_BF16, TOL_F32, err, gpu_fwd, sel_heads, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _ref(inputs, heads=None, S0=None):
+    return oracle.forward(inputs, heads=heads, S0=S0)
+
+
+def _check(y, S, o, ref, heads, tol, S_heads=None):
+    ys = sel_heads(y, heads)
+    os_ = sel_heads(o, heads) if o is not None else None
+    e_y = err(ys, ref["y"])
+    e_o = err(os_, ref["o_raw"]) if os_ is not None else 0.0
+    e_s = err(torch.stack([S[b, h] for (b, h) in heads]), ref["S"]) if S is not None else 0.0
+    assert e_y <= tol and e_o <= tol and e_s <= tol, (e_y, e_o, e_s)
+    return e_y, e_o, e_s
+
+
+def test_tiny_f32_config_all_heads():
+    inp = synth.generate_config("tiny_f32")
+    y, S, o = gpu_fwd(inp)
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_F32)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_f32_shapes_and_chunks_ragged(dk, dv, chunk):
+    shape = synth.GdnShape(B=2, T=157, H=2, dk=dk, dv=dv, chunk=chunk, dtype="f32",
+                           u_low=-5, u_high=-1, seed=dk + dv + chunk)
+    inp = synth.generate(shape)
+    y, S, o = gpu_fwd(inp, chunk=chunk, path="simt")
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_F32)
+
+
+@pytest.mark.parametrize("path", ["auto", "simt"])
+def test_bf16_several_chunks_ragged_tail(path):
+    shape = synth.GdnShape(B=2, T=64 * 5 + 23, H=3, dk=128, dv=128, dtype="bf16",
+                           hot_channels=6, seed=11)
+    inp = synth.generate(shape)
+    y, S, o = gpu_fwd(inp, path=path)
+    heads = oracle.all_heads(2, 3)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
+
+
+def test_state_in_and_in_place_out():
+    shape = synth.GdnShape(B=1, T=130, H=2, dk=64, dv=64, dtype="f32", u_low=-5, u_high=-1, seed=3)
+    inp = synth.generate(shape)
+    S0 = torch.randn(1, 2, 64, 64, generator=torch.Generator().manual_seed(1)) * 0.5
+    d = to_dev(inp)
+    S = S0.cuda()
+    import channel_gated_delta_b200 as gd
+    y, S_out = gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                     d["log_alpha"], gamma_stat=d["gamma_stat"], S_in=S, S_out=S)
+    torch.cuda.synchronize()
+    heads = oracle.all_heads(1, 2)
+    ref = _ref(inp, heads, S0=S0.reshape(2, 64, 64))
+    assert S_out.data_ptr() == S.data_ptr()
+    _check(y.cpu(), S.cpu(), None, ref, heads, TOL_F32)
+
+
+def test_empty_and_single_token():
+    import channel_gated_delta_b200 as gd
+    shape = synth.GdnShape(B=2, T=1, H=2, dk=128, dv=128, dtype="f32", seed=4)
+    inp = synth.generate(shape)
+    S0 = torch.randn(2, 2, 128, 128, generator=torch.Generator().manual_seed(2))
+    y, S, o = gpu_fwd(inp, S_in=S0.cuda())
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, _ref(inp, heads, S0=S0.reshape(4, 128, 128)), heads, TOL_F32)
+    # T = 0: the state passes through unchanged
+    d = to_dev({k: v[:, :0] if v.dim() == 4 else v for k, v in inp.items()})
+    y0, S_out = gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                      d["log_alpha"], S_in=S0.cuda())
+    torch.cuda.synchronize()
+    assert y0.numel() == 0 and torch.equal(S_out.cpu(), S0)
+
+
+def test_split_run_carries_state():
+    shape = synth.GdnShape(B=1, T=300, H=2, dk=128, dv=128, dtype="bf16", seed=5)
+    inp = synth.generate(shape)
+    first = {k: (v[:, :131] if v.dim() == 4 else v) for k, v in inp.items()}
+    second = {k: (v[:, 131:] if v.dim() == 4 else v) for k, v in inp.items()}
+    y1, S1, _ = gpu_fwd(first)
+    y2, S2, _ = gpu_fwd(second, S_in=S1.cuda())
+    heads = oracle.all_heads(1, 2)
+    ref = _ref(inp, heads)
+    assert err(sel_heads(torch.cat([y1, y2], 1), heads), ref["y"]) <= TOL_BF16
+    assert err(torch.stack([S2[b, h] for b, h in heads]), ref["S"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("layer350m_bf16", [(0, 0), (3, 5), (7, 7)]),
+    ("muir1b3_bf16", [(0, 0), (1, 9), (3, 15)]),
+    ("long32k_bf16", [(0, 0), (0, 11)]),
+])
+def test_full_size_configs_sampled_heads(name, heads):
+    """Full workload in the benchmark's launch configuration; the oracle
+    recomputes the sampled heads (heads are independent)."""
+    inp = synth.generate_config(name)
+    y, S, o = gpu_fwd(inp)
+    assert torch.isfinite(y.float()).all()
+    _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
+
+
+def test_decode_after_forward_continues_the_sequence():
+    """Decode steps after a chunked forward equal the forward over the
+    concatenated tokens."""
+    import channel_gated_delta_b200 as gd
+    shape = synth.GdnShape(B=2, T=100, H=2, dk=128, dv=128, dtype="bf16", seed=6)
+    inp = synth.generate(shape)
+    pre = {k: (v[:, :96] if v.dim() == 4 else v) for k, v in inp.items()}
+    _, S, _ = gpu_fwd(pre)
+    S = S.cuda()
+    d = to_dev(inp)
+    ys = []
+    for t in range(96, 100):
+        tok = {k: d[k][:, t].contiguous() for k in ("q", "k", "v", "b", "w", "z", "g", "log_alpha")}
+        ys.append(gd.gdelta_decode_step(tok["q"], tok["k"], tok["v"], tok["b"], tok["w"], tok["z"],
+                                        tok["g"], tok["log_alpha"], S,
+                                        gamma_stat=d["gamma_stat"]).cpu())
+    torch.cuda.synchronize()
+    heads = oracle.all_heads(2, 2)
+    ref = _ref(inp, heads)
+    y_dec = torch.stack(ys, 1)                          # [B,4,H,dv]
+    assert err(sel_heads(y_dec, heads), ref["y"][:, 96:]) <= TOL_BF16
+    assert err(torch.stack([S.cpu()[b, h] for b, h in heads]), ref["S"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("dk,dv,dtype", [(128, 128, "f32"), (64, 128, "f32"), (128, 64, "bf16"),
+                                         (64, 64, "bf16")])
+def test_decode_shapes(dk, dv, dtype):
+    import channel_gated_delta_b200 as gd
+    B, H, steps = 3, 2, 5
+    gen = torch.Generator().manual_seed(dk + dv)
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.3
+    gamma = torch.exp(0.1 * torch.randn(H, dk, generator=gen))
+    S = S0.cuda()
+    heads = oracle.all_heads(B, H)
+    Sref = S0.reshape(B * H, dk, dv).double().numpy()
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    for s in range(steps):
+        inp = synth.decode_step_inputs(s, seed=99, B=B, H=H, dk=dk, dv=dv)
+        if dtype == "f32":
+            inp = {k: v.float() for k, v in inp.items()}
+        d = to_dev(inp)
+        o_raw = torch.empty(B, H, dv, device="cuda")
+        y = gd.gdelta_decode_step(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                  d["log_alpha"], S, gamma_stat=gamma.cuda(), o_raw=o_raw)
+        ref = oracle.decode_steps([inp], Sref, gamma_stat=gamma, heads=heads)
+        Sref = ref["S"]
+        assert err(y.cpu().reshape(B * H, dv), ref["y"][0]) <= tol
+        assert err(o_raw.cpu().reshape(B * H, dv), ref["o_raw"][0]) <= tol
+    assert err(S.cpu().reshape(B * H, dk, dv), Sref) <= tol
+
+
+def test_decode_full_workload_sampled_heads():
+    """Batch 64 x 16 heads, d 128: state from 2048 tokens of the 350M-layer
+    distributions (oracle, sampled heads; other heads start at zero), then
+    1024 consecutive steps on the GPU; the oracle follows the sampled heads."""
+    import channel_gated_delta_b200 as gd
+    D = synth.DECODE
+    B, H, dk, dv = D["B"], D["H"], D["dk"], D["dv"]
+    heads = [(0, 0), (5, 3), (17, 15), (40, 8), (63, 1), (63, 14)]
+    gamma = synth.decode_gamma()
+    S_init = torch.zeros(B, H, dk, dv)
+    Sref = np.zeros((len(heads), dk, dv))
+    by_b = {}
+    for n, (b, h) in enumerate(heads):
+        by_b.setdefault(b, []).append((n, h))
+    for b, lst in by_b.items():
+        tok = synth.decode_init_tokens(b)
+        r = oracle.forward(tok, heads=[(0, h) for _, h in lst])      # S_0 = 0, gamma = 1
+        for (n, h), S_h in zip(lst, r["S"]):
+            Sref[n] = S_h
+            S_init[b, h] = torch.from_numpy(S_h).float()
+    Sref = S_init.double().numpy()[[b for b, _ in heads], [h for _, h in heads]]
+    S = S_init.cuda()
+    gam = gamma.cuda()
+    worst_y = 0.0
+    for s in range(D["steps"]):
+        inp = synth.decode_step_inputs(s)
+        d = to_dev(inp)
+        y = gd.gdelta_decode_step(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                  d["log_alpha"], S, gamma_stat=gam)
+        ref = oracle.decode_steps([inp], Sref, gamma_stat=gamma, heads=heads)
+        Sref = ref["S"]
+        yh = torch.stack([y[b, h] for b, h in heads]).cpu()
+        worst_y = max(worst_y, err(yh, ref["y"][0]))
+    torch.cuda.synchronize()
+    assert worst_y <= TOL_BF16
+    assert err(torch.stack([S.cpu()[b, h] for b, h in heads]), Sref) <= TOL_BF16
