@@ -28,7 +28,8 @@ static int *status_ptr() {
 static bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
 static bool dim_ok(int d) { return d == 64 || d == 128; }
 
-static gdelta_status check_fwd(const gdelta_fwd_args *a) {
+// Shape/dtype/path checks, plus (for a real call) the required pointers.
+static gdelta_status check_fwd(const gdelta_fwd_args *a, bool need_tensors = true) {
     if (!a) return GDELTA_ERR_INVALID_ARG;
     if (a->B < 1 || a->H < 1 || a->T < 0) return GDELTA_ERR_INVALID_ARG;
     if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return GDELTA_ERR_INVALID_ARG;
@@ -37,7 +38,7 @@ static gdelta_status check_fwd(const gdelta_fwd_args *a) {
     const int C = a->chunk == 0 ? 64 : a->chunk;
     if (C != 16 && C != 32 && C != 64) return GDELTA_ERR_UNSUPPORTED;
     if (a->path < GDELTA_PATH_AUTO || a->path > GDELTA_PATH_TC) return GDELTA_ERR_INVALID_ARG;
-    if (a->T > 0) {
+    if (need_tensors && a->T > 0) {
         if (!a->q || !a->k || !a->z || !a->b || !a->v || !a->w || !a->g || !a->log_alpha || !a->y)
             return GDELTA_ERR_INVALID_ARG;
     }
@@ -77,12 +78,12 @@ const char *gdelta_status_string(gdelta_status s) {
 }
 
 int gdelta_fwd_selected_path(const gdelta_fwd_args *args) {
-    if (check_fwd(args) != GDELTA_OK) return -1;
+    if (check_fwd(args, false) != GDELTA_OK) return -1;
     return select_path(args);
 }
 
 size_t gdelta_fwd_workspace_bytes(const gdelta_fwd_args *args) {
-    if (check_fwd(args) != GDELTA_OK) return 0;
+    if (check_fwd(args, false) != GDELTA_OK) return 0;
     return 0;
 }
 

@@ -21,6 +21,22 @@ def err(x, ref) -> float:
     return float(np.max(np.abs(x - ref)) / max(rms, 1e-300))
 
 
+def err_stored(x, ref, storage) -> float:
+    """``err`` for an output stored in a 16-bit float: each element may also
+    carry its storage rounding (half an ulp of the reference value in that
+    format) on top of the computation error.  fp32 outputs use ``err``."""
+    if storage == "f32":
+        return err(x, ref)
+    x = x.detach().cpu().double().numpy() if isinstance(x, torch.Tensor) else np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    mant = {"bf16": 8, "f16": 11}[storage]          # significand bits incl. the implicit one
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 1e-300)))
+    half_ulp = np.ldexp(1.0, (e - mant).astype(np.int64))
+    rms = np.sqrt(np.mean(ref * ref))
+    excess = np.maximum(np.abs(x - ref) - half_ulp, 0.0)
+    return float(np.max(excess) / max(rms, 1e-300))
+
+
 def gpu_fwd(inputs, **kw):
     """Runs the chunked forward through the C ABI; returns CPU tensors."""
     import channel_gated_delta_b200 as gd
