@@ -20,6 +20,7 @@ STATUS_NAMES = {
     4: "GDELTA_ERR_CUDA",
     5: "GDELTA_ERR_TIMEOUT",
     6: "GDELTA_ERR_WORKSPACE",
+    7: "GDELTA_ERR_RANGE",
 }
 GDELTA_F32, GDELTA_BF16 = 0, 1
 PATHS = {"auto": 0, "simt": 1, "tc": 2}

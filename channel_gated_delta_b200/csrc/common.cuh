@@ -29,7 +29,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // Device status codes written by kernels that detect a run-time fault.
-enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1 };
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2 };
 
 struct FwdParams {
     int B, T, H, dk, dv, C;
@@ -58,5 +58,7 @@ cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
 size_t fwd_simt_smem_bytes(int dk, int dv, int C);
 int fwd_simt_chunk(int dk, int dv, int requested);
 cudaError_t launch_state_init(float *S, const float *src, size_t n, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdParams &p, cudaStream_t stream);
+bool fwd_tc_supported(int dtype, int dk, int dv, int chunk);
 
 }  // namespace gdelta

@@ -50,9 +50,10 @@ static gdelta_status check_fwd(const gdelta_fwd_args *a, bool need_tensors = tru
 }
 
 static int select_path(const gdelta_fwd_args *a) {
-    // The tensor-core kernel is not part of this build yet: every shape runs
-    // on the fp32 CUDA-core kernel.
-    if (a->path == GDELTA_PATH_TC) return -1;
+    const int C = a->chunk == 0 ? 64 : a->chunk;
+    const bool tc_ok = fwd_tc_supported(a->dtype, a->dk, a->dv, C);
+    if (a->path == GDELTA_PATH_TC) return tc_ok ? GDELTA_PATH_TC : -1;
+    if (a->path == GDELTA_PATH_AUTO && tc_ok) return GDELTA_PATH_TC;
     return GDELTA_PATH_SIMT;
 }
 
@@ -73,6 +74,7 @@ const char *gdelta_status_string(gdelta_status s) {
         case GDELTA_ERR_CUDA: return "CUDA error";
         case GDELTA_ERR_TIMEOUT: return "device-side bounded wait ran out";
         case GDELTA_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDELTA_ERR_RANGE: return "a value left the tensor-core path's fp16 operand range";
     }
     return "unknown status";
 }
@@ -120,6 +122,10 @@ gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     p.la = a->log_alpha; p.gs = a->gamma_stat; p.S_in = a->S_in; p.S_out = a->S_out;
     p.y = a->y; p.o_raw = a->o_raw; p.eps = a->eps;
     p.status = status_ptr();
+    if (path == GDELTA_PATH_TC) {
+        p.C = 64;
+        return launch_fwd_tc(p, s) == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
+    }
     p.C = fwd_simt_chunk(a->dk, a->dv, a->chunk == 0 ? 64 : a->chunk);
     if (p.C == 0) return GDELTA_ERR_UNSUPPORTED;
     return launch_fwd_simt(p, a->dtype, s) == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
@@ -156,7 +162,8 @@ gdelta_status gdelta_get_last_device_error(void *stream) {
         const int zero = 0;
         cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
     }
-    return v == kDevOk ? GDELTA_OK : GDELTA_ERR_TIMEOUT;
+    if (v == kDevOk) return GDELTA_OK;
+    return v == kDevRange ? GDELTA_ERR_RANGE : GDELTA_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -62,7 +62,9 @@ typedef enum gdelta_status {
     GDELTA_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
     GDELTA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     GDELTA_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (device status) */
-    GDELTA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+    GDELTA_ERR_WORKSPACE = 6,     /* workspace missing or smaller than required */
+    GDELTA_ERR_RANGE = 7          /* device status: an fp16 tensor-core operand (state, erase
+                                     projection or scaled key/query) exceeded 6e4 in magnitude */
 } gdelta_status;
 
 typedef enum gdelta_dtype {
@@ -175,7 +177,9 @@ GDELTA_API gdelta_status gdelta_decode_step(const gdelta_decode_args *args, void
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns GDELTA_OK, GDELTA_ERR_TIMEOUT (a kernel's bounded
- * wait ran out) or GDELTA_ERR_CUDA (the synchronisation itself failed).
+ * wait ran out), GDELTA_ERR_RANGE (the tensor-core path met an operand
+ * outside its fp16 range; its results are unreliable, rerun with
+ * GDELTA_PATH_SIMT) or GDELTA_ERR_CUDA (the synchronisation itself failed).
  */
 GDELTA_API gdelta_status gdelta_get_last_device_error(void *stream);
 

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_abi_version_and_status_strings(lib):
     assert lib.gdelta_abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         s = lib.gdelta_status_string(code)
         assert s and s != b"unknown status"
     assert lib.gdelta_status_string(99) == b"unknown status"

@@ -206,3 +206,62 @@ def test_decode_full_workload_sampled_heads():
     torch.cuda.synchronize()
     assert worst_y <= TOL_BF16
     assert err(torch.stack([S.cpu()[b, h] for b, h in heads]), Sref) <= TOL_BF16
+
+
+# --------------------------------------------------------------------------
+# Tensor-core path (tcgen05, fp16 operands, fp32 accumulation)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 5, 64, 65, 200, 64 * 7 + 9])
+def test_tc_ragged_lengths(T):
+    shape = synth.GdnShape(B=2, T=T, H=2, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=40 + T)
+    inp = synth.generate(shape)
+    y, S, o = gpu_fwd(inp, path="tc")
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
+
+
+@pytest.mark.parametrize("u", [(-3.0, 0.0), (0.0, 2.0), (2.0, 3.5)])
+def test_tc_fast_decay_shortens_chunks(u):
+    """Decays fast enough that a 64-token chunk's log-decay span exceeds the
+    fp16 operand budget: the kernel shortens chunks (down to one token)."""
+    shape = synth.GdnShape(B=1, T=300, H=2, dk=128, dv=128, dtype="bf16", u_low=u[0], u_high=u[1], seed=7)
+    inp = synth.generate(shape)
+    y, S, o = gpu_fwd(inp, path="tc")
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
+
+
+def test_tc_state_in_and_in_place():
+    import channel_gated_delta_b200 as gd
+    shape = synth.GdnShape(B=2, T=150, H=3, dk=128, dv=128, dtype="bf16", seed=8)
+    inp = synth.generate(shape)
+    S0 = torch.randn(2, 3, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.3
+    d = to_dev(inp)
+    S = S0.cuda()
+    y, _ = gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"],
+                                 gamma_stat=d["gamma_stat"], S_in=S, S_out=S, path="tc")
+    torch.cuda.synchronize()
+    assert gd.gdelta_get_last_device_error() == 0
+    heads = oracle.all_heads(2, 3)
+    ref = _ref(inp, heads, S0=S0.reshape(6, 128, 128))
+    _check(y.cpu(), S.cpu(), None, ref, heads, TOL_BF16)
+
+
+def test_tc_matches_simt_path():
+    shape = synth.GdnShape(B=1, T=256, H=4, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=9)
+    inp = synth.generate(shape)
+    y1, S1, o1 = gpu_fwd(inp, path="tc")
+    y2, S2, o2 = gpu_fwd(inp, path="simt")
+    assert err(o1, o2.double().numpy()) <= TOL_BF16
+    assert err(S1, S2.double().numpy()) <= TOL_BF16
+
+
+def test_tc_rejects_unsupported_shapes():
+    import channel_gated_delta_b200 as gd
+    shape = synth.GdnShape(B=1, T=64, H=1, dk=64, dv=64, dtype="bf16", seed=1)
+    d = to_dev(synth.generate(shape))
+    with pytest.raises(gd.GdeltaError):
+        gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], path="tc")
+    assert gd.gdelta_fwd_selected_path(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                       d["log_alpha"]) == "simt"
