@@ -58,7 +58,8 @@ cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
 size_t fwd_simt_smem_bytes(int dk, int dv, int C);
 int fwd_simt_chunk(int dk, int dv, int requested);
 cudaError_t launch_state_init(float *S, const float *src, size_t n, cudaStream_t stream);
-cudaError_t launch_fwd_tc(const FwdParams &p, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdParams &p, void *workspace, cudaStream_t stream);
+size_t fwd_tc_workspace_bytes(int B, int H, int T);
 bool fwd_tc_supported(int dtype, int dk, int dv, int chunk);
 
 }  // namespace gdelta

@@ -86,6 +86,7 @@ int gdelta_fwd_selected_path(const gdelta_fwd_args *args) {
 
 size_t gdelta_fwd_workspace_bytes(const gdelta_fwd_args *args) {
     if (check_fwd(args, false) != GDELTA_OK) return 0;
+    if (select_path(args) == GDELTA_PATH_TC && args->T > 0) return fwd_tc_workspace_bytes(args->B, args->H, args->T);
     return 0;
 }
 
@@ -124,7 +125,9 @@ gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     p.status = status_ptr();
     if (path == GDELTA_PATH_TC) {
         p.C = 64;
-        return launch_fwd_tc(p, s) == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
+        const size_t need = fwd_tc_workspace_bytes(a->B, a->H, a->T);
+        if (!a->workspace || a->workspace_bytes < need) return GDELTA_ERR_WORKSPACE;
+        return launch_fwd_tc(p, a->workspace, s) == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
     }
     p.C = fwd_simt_chunk(a->dk, a->dv, a->chunk == 0 ? 64 : a->chunk);
     if (p.C == 0) return GDELTA_ERR_UNSUPPORTED;
