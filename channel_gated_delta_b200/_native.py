@@ -34,6 +34,7 @@ EXPORTED = (
     "gdelta_fwd_selected_path",
     "gdelta_state_init",
     "gdelta_fwd_chunked",
+    "gdelta_fwd_chunked_noalloc",
     "gdelta_decode_step",
     "gdelta_get_last_device_error",
 )
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH):
                                       ctypes.c_int32, _fp, _vp]
     lib.gdelta_fwd_chunked.restype = ctypes.c_int
     lib.gdelta_fwd_chunked.argtypes = [ctypes.POINTER(FwdArgs), _vp]
+    lib.gdelta_fwd_chunked_noalloc.restype = ctypes.c_int
+    lib.gdelta_fwd_chunked_noalloc.argtypes = [ctypes.POINTER(FwdArgs), _vp]
     lib.gdelta_decode_step.restype = ctypes.c_int
     lib.gdelta_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
     lib.gdelta_get_last_device_error.restype = ctypes.c_int

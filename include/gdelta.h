@@ -171,6 +171,31 @@ GDELTA_API gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32
 /* Chunked forward; see gdelta_fwd_args. */
 GDELTA_API gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *args, void *stream);
 
+/*
+ * Chunked forward that allocates nothing and needs no workspace argument.
+ * The pages describe nothing like it: it exists for callers that cannot
+ * allocate device memory when they run the forward -- code inside a runtime
+ * that plans all device memory in advance, or latency-critical code that must
+ * not call cudaMalloc (it synchronises the device and can fail).  The scratch
+ * the tensor-core path needs lives in a fixed 32 MiB device array inside the
+ * library, which every device that loads the library holds until the process
+ * exits; args->workspace and args->workspace_bytes are ignored.
+ *
+ *  - Limit: gdelta_fwd_workspace_bytes(args) must not exceed 32 MiB (105 KiB
+ *    per 64-token window of each batch row and head, plus one int per window:
+ *    311 windows, e.g. B = 1, H = 16, T <= 1216).  Larger problems return
+ *    GDELTA_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address (a CUDA
+ *    runtime call); make that first call before capturing any stream.
+ *  - Every call uses the same array.  Each call writes every scratch entry it
+ *    later reads, so nothing needs clearing between calls, but two calls
+ *    whose kernels overlap on the GPU (different streams, no ordering) race
+ *    on the array and give wrong results: order them on one stream.
+ *  - Otherwise identical to gdelta_fwd_chunked (same arguments, results and
+ *    status codes).
+ */
+GDELTA_API gdelta_status gdelta_fwd_chunked_noalloc(const gdelta_fwd_args *args, void *stream);
+
 /* One decode step; see gdelta_decode_args. */
 GDELTA_API gdelta_status gdelta_decode_step(const gdelta_decode_args *args, void *stream);
 
