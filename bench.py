@@ -288,6 +288,7 @@ def run_ours(args, rank, local, world):
         "config": {
             "workload": f"{WORKLOAD}: B{B} T{T} H{H} dk=dv={dk} chunk {C}, bf16 tokens, fp32 log-decay and state",
             "step": "state_init + fwd_chunked + 1 decode step (all heads)",
+            "kernels_per_step": 4 if path == "tc" else 3,
             "tokens_per_step_per_gpu": tok_per_step,
             "kernel_path": path,
             "workspace_bytes": ws_bytes,
@@ -309,7 +310,8 @@ def run_ours(args, rank, local, world):
         },
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        # state init + decode + forward (the tensor-core forward is two kernels)
+        "gpu_launches": (4 if path == "tc" else 3) * args.steps,
         "clocks": clk,
         "decode": dec,
     }
