@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
 
     const size_t sbase = (size_t)head * kDK * kDV;
     bool first = true;
+    bool prefetched = false;                      // the current window's record is already in flight
     for (int w = 0; w < p.NW && flags[0] == 0; ++w) {
     const int wend = min(T, kC * (w + 1));
     // windows with precomputed chunk tiles (intra kernel) take the fast path;
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
         int n;
         if (fast) {
             const uint8_t *rec = p.ws + ((size_t)head * p.NW + w) * kWinBytes;
-            if (tid == 0) {
+            if (tid == 0 && !prefetched) {
                 tc::fence_proxy_async();
                 tc::mbar_arrive_expect_tx(s_tbar, kWinBytes - kWinPad);
                 tc::bulk_g2s(s_ap, rec + kWinAP, 128 * 256, s_tbar);
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
             __syncthreads();
             if (flags[0]) break;
             n = wend - t0;
+            prefetched = false;
         } else {
             // ---- A: loads, cumulative log-decay, span, chunk length.
             // Warp w owns tokens [8w, 8w+8); lane l owns key channels [4l, 4l+4)
@@ -674,6 +676,27 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
             tc::mma_commit(s_mbar);
         }
         if (!wait_mma()) break;
+        // the chunk's tiles are free: keep its decay factor, then start the
+        // bulk copy of the next window's record so it overlaps the epilogue
+        if (tid < kDK) fprev[tid] = fcv[tid];
+        {
+            const bool next_fast = t0 + n == wend && w + 1 < p.NW && p.ws != nullptr &&
+                                   p.wflags[(size_t)head * p.NW + w + 1] == 0;
+            __syncthreads();
+            if (next_fast) {
+                if (tid == 0) {
+                    const uint8_t *nrec = p.ws + ((size_t)head * p.NW + w + 1) * kWinBytes;
+                    tc::fence_proxy_async();
+                    tc::mbar_arrive_expect_tx(s_tbar, kWinBytes - kWinPad);
+                    tc::bulk_g2s(s_ap, nrec + kWinAP, 128 * 256, s_tbar);
+                    tc::bulk_g2s(s_bp, nrec + kWinBP, 128 * 256, s_tbar);
+                    tc::bulk_g2s(s_anab, nrec + kWinANAB, 192 * 128, s_tbar);
+                    tc::bulk_g2s(s_vh, nrec + kWinVH, 64 * 2 * kDV, s_tbar);
+                    tc::bulk_g2s(tc::smem_u32(ecv), nrec + kWinVEC, 2 * 128 * 4, s_tbar);
+                }
+                prefetched = true;
+            }
+        }
 
         // ---- L: O (rows 64-127) -> RMSNorm over the head's d_v, gate, store
         {
@@ -715,7 +738,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
                     }
                 }
             }
-            if (tid < kDK) fprev[tid] = fcv[tid];
         }
         tc::fence_before_sync();
         __syncthreads();
@@ -723,6 +745,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
         t0 += n;
     }
     }
+
+    // a prefetch still in flight (the loop ended early) completes before exit
+    if (prefetched) tc::mbar_wait(s_tbar, tphase);
 
     // ---- S_out = Diag(f) X
     if (flags[0] == 0 && p.S_out && T > 0) {
