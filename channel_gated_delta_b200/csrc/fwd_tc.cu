@@ -47,6 +47,49 @@ constexpr float kSpanMax = 12.f;
 constexpr int kThreads = 256;
 constexpr int kLW = 68;       // row stride (floats) of the fp32 L / T^-1 matrix
 constexpr int kYS = 36;       // row stride (floats) of the merge buffer
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).  With
+// log-decays pre-scaled by log2(e), e^x = 2^(x log2 e) costs one instruction.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2 sigmoid(z) = 2 / (1 + e^-z); the exponent is clamped so that the sum stays finite.
+__device__ __forceinline__ float two_sigmoid_fast(float z) {
+    return __fdividef(2.f, 1.f + ex2(fminf(-z * kLog2e, 126.f)));
+}
+
+// Warp reduce-scatter of 16 per-lane partial sums: afterwards lane l holds the
+// sum over all 32 lanes of value 8 b4 + 4 b3 + 2 b2 + b1 (b_i = bit i of l),
+// in 16 shuffles instead of the 80 of sixteen separate butterflies.
+__device__ __forceinline__ float reduce_scatter16(const float (&v)[16], int lane) {
+    float w8[8], w4[4], w2[2];
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float keep = b4 ? v[8 + j] : v[j], send = b4 ? v[j] : v[8 + j];
+        w8[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float keep = b3 ? w8[4 + j] : w8[j], send = b3 ? w8[j] : w8[4 + j];
+        w4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float keep = b2 ? w4[2 + j] : w4[j], send = b2 ? w4[j] : w4[2 + j];
+        w2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    float w1;
+    {
+        const float keep = b1 ? w2[1] : w2[0], send = b1 ? w2[0] : w2[1];
+        w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
+}
 
 // shared-memory map (bytes); tiles are 1024-byte aligned
 template <int DVC>
@@ -849,7 +892,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
     };
 
     do {
-        // ---- loads (whole 256-byte token rows per instruction) and the log-decay scan
+        // ---- loads (whole 256-byte token rows per instruction) and the log-decay
+        // scan, in log2 units (Lambda * log2 e) so that every decay factor is one ex2
         const int tb = 8 * warp, c4 = 4 * lane;
         float la[8][4];
         uint2 kq[8][4];
@@ -860,7 +904,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             const size_t gk = (((size_t)bb * T + t0 + t) * H + h) * kDK + c4;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (in) x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
-            la[u][0] = x.x; la[u][1] = x.y; la[u][2] = x.z; la[u][3] = x.w;
+            la[u][0] = x.x * kLog2e; la[u][1] = x.y * kLog2e; la[u][2] = x.z * kLog2e; la[u][3] = x.w * kLog2e;
             kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
             kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
             kq[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
@@ -900,24 +944,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             float m = 0.f;
 #pragma unroll
             for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, spanred[ww]);
-            if (m > kSpanMax) {                       // the chain kernel takes this window
+            if (m > kSpanMax * kLog2e) {              // the chain kernel takes this window
                 if (tid == 0) wflags[wi] = 1;
                 break;
             }
         }
         const int n = wend - t0;
-        uint2 vw[8][2];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = tb + u;
-            const bool in = t0 + t < wend;
-            const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + c4;
-            vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-            vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
-        }
 
-        // ---- operand tiles: P operands to shared memory; Qp, Kc, K^c, V^ and
-        // the pivot vectors straight to the window record
+        // ---- operand tiles: P operands to shared memory; Qp, Kc, K^c and the
+        // pivot vectors straight to the window record
         {
             const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
             const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
@@ -929,22 +964,21 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             }
             if (warp == 0) {
                 float4 *rv = reinterpret_cast<float4 *>(rec + kWinVEC);
-                rv[lane] = make_float4(__expf(cpiv[0]), __expf(cpiv[1]), __expf(cpiv[2]), __expf(cpiv[3]));
-                rv[32 + lane] = make_float4(__expf(lnv[0] - cpiv[0]), __expf(lnv[1] - cpiv[1]), __expf(lnv[2] - cpiv[2]),
-                                            __expf(lnv[3] - cpiv[3]));
+                rv[lane] = make_float4(ex2(cpiv[0]), ex2(cpiv[1]), ex2(cpiv[2]), ex2(cpiv[3]));
+                rv[32 + lane] = make_float4(ex2(lnv[0] - cpiv[0]), ex2(lnv[1] - cpiv[1]), ex2(lnv[2] - cpiv[2]),
+                                            ex2(lnv[3] - cpiv[3]));
             }
+            float dg[16];                             // [u]: q~.k, [8+u]: q~.(b*k) of token tb+u, this lane's channels
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = tb + u;
                 const bool live = t < n;
-                float kk[4], qq[4], zz[4], bv[4], vv[4], ww4[4];
+                float kk[4], qq[4], zz[4], bv[4];
                 {
                     const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][0]);
                     const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][1]);
                     const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][2]);
                     const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][3]);
-                    const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
-                    const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         float2 f;
@@ -952,19 +986,17 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                         f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
                         f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
                         f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
-                        f = __bfloat1622float2(hv[e]); vv[2 * e] = f.x; vv[2 * e + 1] = f.y;
-                        f = __bfloat1622float2(hw[e]); ww4[2 * e] = f.x; ww4[2 * e + 1] = f.y;
                     }
                 }
-                float kp[4], kc[4], khc[4], qp[4], vh[4];
+                float kp[4], kc[4], khc[4], qp[4];
                 float dq = 0.f, db = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const float lam = live ? la[u][c] : lnv[c];
                     const float d = lam - cpiv[c];
-                    const float ep = __expf(d), em = __expf(-d);
+                    const float ep = ex2(d), em = ex2(-d);
                     const float kv = live ? kk[c] : 0.f;
-                    const float qt = live ? qq[c] * gq[c] * (2.f / (1.f + __expf(-zz[c]))) : 0.f;
+                    const float qt = live ? qq[c] * gq[c] * two_sigmoid_fast(zz[c]) : 0.f;
                     const float kh = bv[c] * kv;
                     dq += qt * kv;
                     db += qt * kh;
@@ -972,19 +1004,11 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                     kc[c] = kv * em;
                     khc[c] = kh * em;
                     qp[c] = qt * ep;
-                    vh[c] = live ? vv[c] * ww4[c] : 0.f;
                 }
                 range_max = fmaxf(range_max, fmaxf(fmaxf(maxabs(kp, 4), maxabs(kc, 4)),
                                                    fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    dq += __shfl_xor_sync(0xffffffffu, dq, o);
-                    db += __shfl_xor_sync(0xffffffffu, db, o);
-                }
-                if (lane == 0) {
-                    diagq[t] = dq;
-                    diagb[t] = db;
-                }
+                dg[u] = dq;
+                dg[8 + u] = db;
                 const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
                 const uint2 ukp = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
                 const uint2 uqp = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
@@ -997,9 +1021,23 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 *(uint2 *)(rec + kWinAP + off_b) = uqp;
                 *(uint2 *)(rec + kWinBP + off_t) = ukc;
                 *(uint2 *)(rec + kWinBP + off_b) = ukh;
-                *(uint2 *)(rec + kWinVH + tc::tile_off(64, t, c4)) =
-                    make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
             }
+            // the exact diagonals q~_t.k_t and q~_t.(b*k)_t of Aq / Bq
+            const float dsum = reduce_scatter16(dg, lane);
+            if ((lane & 1) == 0) {
+                const int vi = (lane >> 1) & 15;
+                (vi < 8 ? diagq : diagb)[tb + (vi & 7)] = dsum;
+            }
+        }
+        // value side: loads issued now, consumed while the P product runs
+        uint2 vw[8][2];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = tb + u;
+            const bool in = t0 + t < wend;
+            const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + c4;
+            vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+            vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
         }
         tc::fence_proxy_async();
         __syncthreads();
@@ -1012,25 +1050,50 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 tc::mma_f16(tmem, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id, ks > 0);
             tc::mma_commit(s_mbar);
         }
+        // V^ = w*v -> window record (the identity padding past n is zero)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = tb + u;
+            const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
+            const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
+            float vh[4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float2 fv = __bfloat1622float2(hv[e]), fw = __bfloat1622float2(hw[e]);
+                vh[2 * e] = fv.x * fw.x;
+                vh[2 * e + 1] = fv.y * fw.y;
+            }
+            *(uint2 *)(rec + kWinVH + tc::tile_off(64, t, c4)) =
+                make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
+        }
         if (!wait_mma()) break;
 
-        // ---- masks; M -> MM (shared), L -> fp32 (over BP), Aq / Bq -> record
+        // ---- masks; M -> MM (shared), L -> fp32 (over BP), Aq / Bq -> record.
+        // This warp's rows are tokens t in [32 tb2, 32 tb2 + 32): column block hf
+        // below the diagonal block is kept whole, above it zeroed, and only the
+        // diagonal block is masked element by element.
         {
             const int t = row & 63;
             const bool upper = row < 64;
+            const int tb2 = warp & 1;
             float v[2][32];
             tc::tmem_ld32x2(tmem + lane_base + 64 * colhalf, tmem + lane_base + 64 * colhalf + 32, v[0], v[1]);
             // all warps have read P; BP may now be overwritten with L
             tc::fence_before_sync();
             __syncthreads();
+            const float dv_t = upper ? 0.f : (colhalf == 0 ? diagq[t] : diagb[t]);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
+                if (hf > tb2) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int s = 32 * hf + i;
-                    const bool keep = upper ? (s < t) : (s <= t);
-                    if (!keep) v[hf][i] = 0.f;
-                    if (!upper && s == t) v[hf][i] = colhalf == 0 ? diagq[t] : diagb[t];
+                    for (int i = 0; i < 32; ++i) v[hf][i] = 0.f;
+                } else if (hf == tb2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const bool keep = upper ? (i < lane) : (i <= lane);
+                        if (!keep) v[hf][i] = 0.f;
+                        if (!upper && i == lane) v[hf][i] = dv_t;
+                    }
                 }
                 if (upper && colhalf == 1) {
                     float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
