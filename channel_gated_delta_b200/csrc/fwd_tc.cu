@@ -45,6 +45,7 @@ constexpr int kDK = 128;      // key channels
 constexpr int kDV = 128;      // value channels of a head
 constexpr float kSpanMax = 12.f;
 constexpr int kThreads = 256;
+constexpr int kChainThreads = 384;   // chain kernel: 8 state warps, 2 idle, 2 readout warps
 constexpr int kLW = 68;       // row stride (floats) of the fp32 L / T^-1 matrix
 constexpr int kYS = 36;       // row stride (floats) of the merge buffer
 constexpr float kLog2e = 1.4426950408889634f;
@@ -91,27 +92,35 @@ __device__ __forceinline__ float reduce_scatter16(const float (&v)[16], int lane
     return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
 }
 
-// shared-memory map (bytes); tiles are 1024-byte aligned
-template <int DVC>
-struct Smem {
-    static constexpr int AP = 0;                          // [Kp | W' ; Qp]  128 x 128 fp16
-    static constexpr int BP = AP + 128 * 256;             // [Kc ; K^c]      128 x 128
-    static constexpr int TI = BP + 128 * 256;             // T^-1             64 x 64
-    static constexpr int MM = TI + 64 * 128;              // M                64 x 64
-    static constexpr int ANAB = MM + 64 * 128;            // [N ; Aq ; Bq]   192 x 64
-    static constexpr int VH = ANAB + 192 * 128;           // V^               64 x DVC
-    static constexpr int SC = VH + 64 * 2 * DVC;          // S_c             128 x DVC
-    static constexpr int RR = SC + 128 * 2 * DVC;         // R                64 x DVC
-    static constexpr int GS = RR + 64 * 2 * DVC;          // output gate g (bf16 [64][DVC])
-    static constexpr int LW = GS + 64 * 2 * DVC;          // fp32 L, then T^-1   [64][kLW]
-    static constexpr int YB = LW + 64 * kLW * 4;          // fp32 merge buffer  [32][kYS]
-    static constexpr int WT = YB + 32 * kYS * 4;          // fp32 per-warp log-decay totals [8][128]
-    static constexpr int PR = WT + 8 * 128 * 4;           // fp32 Lambda at the probe tokens [7][128]
-    static constexpr int VEC = PR + 8 * 128 * 4;          // fp32 vectors
-    static constexpr int nvec = 8 * 128;
-    static constexpr int PART = VEC + nvec * 4;           // fp32 [64][2] RMS partial sums
-    static constexpr int MISC = PART + 64 * 2 * 4;        // mbarrier, TMEM slot, flags
-    static constexpr int TOTAL = MISC + 64;
+// Chain-kernel shared-memory map (bytes; tiles 1024-byte aligned).  Two window
+// buffers, each holding one window record in the record's own byte layout
+// (V^ restricted to this CTA's 64 value columns): while window w runs from one
+// buffer, the record of window w+1 is already arriving in the other.  A window
+// processed in shorter chunks (decay span too large for one 64-token chunk)
+// builds its tiles in its own buffer and uses the other one as scratch.
+struct ChainSmem {
+    static constexpr int AP = 0;                         // [W' ; Qp] (shorter chunks: [Kp ; Qp]) 128 x 128 fp16
+    static constexpr int BP = AP + 128 * 256;            // [Kc ; K^c]                            128 x 128
+    static constexpr int ANAB = BP + 128 * 256;          // [N ; Aq ; Bq]                         192 x 64
+    static constexpr int VH = ANAB + 192 * 128;          // V^, this CTA's value columns           64 x 64
+    static constexpr int EV = VH + 64 * 128;             // fp32 e^c [128], e^{Lambda_{n-1} - c} [128]
+    static constexpr int BUF = EV + 1024;                // one window buffer
+    // scratch of the shorter-chunk path, inside the other window buffer
+    static constexpr int TI = 0;                         // T^-1  64 x 64 fp16
+    static constexpr int MM = TI + 64 * 128;             // M     64 x 64 fp16
+    static constexpr int LW = MM + 64 * 128;             // fp32 L, then T^-1   [64][kLW]
+    static constexpr int YB = LW + 64 * kLW * 4;         // fp32 merge buffer   [32][kYS]
+    static constexpr int WT = YB + 32 * kYS * 4;         // fp32 per-warp log-decay totals [8][128]
+    static constexpr int PR = WT + 8 * 128 * 4;          // fp32 Lambda at the probe tokens [7][128]
+    static constexpr int XV = PR + 8 * 128 * 4;          // fp32 span maxima [64], exact diagonals [2][64]
+    static_assert(XV + 192 * 4 <= BUF, "shorter-chunk scratch fits in a window buffer");
+    // shared by all windows
+    static constexpr int SC = 2 * BUF;                   // S_c  128 x 64 fp16
+    static constexpr int RR = SC + 128 * 128;            // R     64 x 64 fp16
+    static constexpr int VEC = RR + 64 * 128;            // fp32 fprev [128], gamma_stat [128]
+    static constexpr int PART = VEC + 256 * 4;           // fp32 peer's row sums [2][64], int peer flags [2]
+    static constexpr int MISC = PART + 1536;             // 11 mbarriers, TMEM slot, flags, chunk info
+    static constexpr int TOTAL = MISC + 256;
 };
 
 // Per-window record written by the intra kernel: the chunk's operand tiles in
@@ -122,14 +131,15 @@ constexpr int kWinBP = kWinAP + 128 * 256;    // [Kc ; K^c]      128 x 128
 constexpr int kWinANAB = kWinBP + 128 * 256;  // [N ; Aq ; Bq]   192 x 64
 constexpr int kWinVH = kWinANAB + 192 * 128;  // V^               64 x 128
 constexpr int kWinVEC = kWinVH + 64 * 256;    // e^c, e^{Lambda_{n-1} - c}
-constexpr int kWinPad = 1024 - 2 * 128 * 4;   // padding to a 1 KB multiple
 constexpr int kWinBytes = kWinVEC + 1024;
 
-// TMEM columns
-constexpr uint32_t kTmP = 0;       // P (128 x 128), later [R; O] (128 x DVC)
-constexpr uint32_t kTmW = 128;     // W' (M=64, 128 columns)
-constexpr uint32_t kTmN = 256;     // N  (M=64, 64 columns)
-constexpr uint32_t kTmX = 384;     // state accumulator X (128 x DVC)
+// Chain-kernel TMEM columns
+constexpr uint32_t kTmP = 0;       // shorter chunks: P (128 x 128)
+constexpr uint32_t kTmW = 128;     // shorter chunks: W' (M=64, 128 columns)
+constexpr uint32_t kTmN = 256;     // shorter chunks: N  (M=64, 64 columns)
+constexpr uint32_t kTmX = 320;     // state accumulator X (128 x 64)
+constexpr uint32_t kTmRO = 384;    // [R; O] (128 x 64)
+constexpr int kDVC = 64;           // value columns per chain CTA; a cluster of two covers d_v = 128
 
 struct TcParams {
     int B, T, H;
@@ -173,6 +183,10 @@ __device__ __forceinline__ void store_row32(uint8_t *tile, int R, int r, int col
         *(uint4 *)(tile + tc::tile_chunk_off(R, r, col / 8 + q4)) = pack8(v + 8 * q4);
 }
 
+// Barrier of warps 0-7 (named barrier 1): the whole intra-kernel CTA, the
+// state warps of the chain kernel.
+__device__ __forceinline__ void main_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // One merge level of the divide-and-conquer inverse, block size BS (pairs of
 // BS x BS blocks along the diagonal of the 64 x 64 matrix in lw).
 template <int BS>
@@ -191,7 +205,7 @@ __device__ __forceinline__ void merge_level(float *lw, float *yb, int tid) {
         }
         *reinterpret_cast<float4 *>(yb + (pr * BS + i) * kYS + j0) = acc;
     }
-    __syncthreads();
+    main_sync();
     if (tid < NTASK) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *drow = lw + (oo + BS + i) * kLW + oo + BS;
@@ -203,569 +217,676 @@ __device__ __forceinline__ void merge_level(float *lw, float *yb, int tid) {
         }
         *reinterpret_cast<float4 *>(lw + (oo + BS + i) * kLW + oo + j0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
-    __syncthreads();
+    main_sync();
 }
 
 }  // namespace
 
-template <int DVC>
-__global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
-    using L = Smem<DVC>;
+// ---------------------------------------------------------------------------
+// Chain kernel: a cluster of two CTAs per (batch, head); CTA r owns value
+// columns [64 r, 64 r + 64) of the state, which stays in TMEM (fp32) for the
+// whole sequence.  Value columns of the recurrence are independent, so the
+// two CTAs share nothing but the RMS norm of the readout: per chunk they
+// exchange per-token sums of squares through distributed shared memory.
+// Windows whose tiles the intra kernel precomputed are bulk-copied one window
+// ahead; a flagged window (decay span too large for one 64-token chunk) is
+// processed here in shorter chunks.
+//
+// Warp roles: warps 0-7 run the state recurrence (operand staging, MMA issue,
+// R readout); warps 10-11 (TMEM lanes 64-127, the readout rows) take each
+// chunk's O out of TMEM and run the RMS exchange, gate and stores while the
+// state recurrence moves on to the next chunk.  [R; O] alternates between two
+// TMEM slots; warps 8-9 have no role.
+// ---------------------------------------------------------------------------
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
+    using L = ChainSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int head = blockIdx.x;                 // b * H + h
+    const uint32_t crank = tc::cluster_ctarank();
+    const int head = blockIdx.x >> 1;            // b * H + h
     const int bb = head / p.H, h = head % p.H;
     const int T = p.T, H = p.H;
-    const int dv0 = 0;                            // first value column of this CTA
+    const int dv0 = kDVC * (int)crank;           // first value column of this CTA
 
-    float *lw = (float *)(sm + L::LW);
-    float *yb = (float *)(sm + L::YB);
-    float *wtot = (float *)(sm + L::WT);
-    float *probe = (float *)(sm + L::PR);
-    float *vec = (float *)(sm + L::VEC);
-    float *ecv = vec + 128, *fcv = vec + 256, *fprev = vec + 384, *gsv = vec + 512;
-    float *spanred = vec + 640;                   // [8 warps][8]
-    float *diagq = vec + 768, *diagb = vec + 896; // exact q~_t.k_t and q~_t.(b*k)_t
-    float *part = (float *)(sm + L::PART);
-    __nv_bfloat16 *gsm = (__nv_bfloat16 *)(sm + L::GS);
+    float *fprev = (float *)(sm + L::VEC), *gsv = fprev + 128;
+    // mbarriers: [0] MMA, [1..2] record buffers, [3..4] exchange slots, [5..6] chunk info,
+    // [7..8] O ready, [9..10] O slot free
     uint64_t *mbar = (uint64_t *)(sm + L::MISC);
-    uint32_t *tslot = (uint32_t *)(sm + L::MISC + 8);
-    int *flags = (int *)(sm + L::MISC + 16);      // [0] abort, [1] chosen n, [2] log2 of the chunk
-    uint64_t *tbar = (uint64_t *)(sm + L::MISC + 32);
-    const uint32_t s_ap = tc::smem_u32(sm + L::AP), s_bp = tc::smem_u32(sm + L::BP);
-    const uint32_t s_ti = tc::smem_u32(sm + L::TI), s_mm = tc::smem_u32(sm + L::MM);
-    const uint32_t s_anab = tc::smem_u32(sm + L::ANAB), s_vh = tc::smem_u32(sm + L::VH);
+    uint32_t *tslot = (uint32_t *)(sm + L::MISC + 88);
+    float *peer = (float *)(sm + L::PART);        // [2][64] the peer's per-row sums
+    int *pflag = (int *)(sm + L::PART + 512);     // [2] the peer's abort flags
+    volatile int *flags = (volatile int *)(sm + L::MISC + 96);  // [0] local abort, [1] chosen n, [2] log2 of the chunk, [3] agreed abort
+    int *info = (int *)(sm + L::MISC + 112);      // per O slot: t0, n, done
+    const uint32_t s_mbar = tc::smem_u32(mbar), s_rbar = s_mbar + 8, s_xbar = s_mbar + 24;
+    const uint32_t s_ibar = s_mbar + 40, s_obar = s_mbar + 56, s_fbar = s_mbar + 72;
+    const uint32_t peer_rank = crank ^ 1u;
+    const uint32_t r_peer = tc::mapa(tc::smem_u32(peer), peer_rank);
+    const uint32_t r_pflag = tc::mapa(tc::smem_u32(pflag), peer_rank);
+    const uint32_t r_xbar = tc::mapa(s_xbar, peer_rank);
     const uint32_t s_sc = tc::smem_u32(sm + L::SC), s_rr = tc::smem_u32(sm + L::RR);
-    const uint32_t s_mbar = tc::smem_u32(mbar), s_tbar = tc::smem_u32(tbar);
 
-    // ---- set-up: TMEM, mbarrier, per-head vectors
+    // ---- set-up: TMEM, mbarriers, per-head vectors; the peer's barriers exist before first use
     if (warp == 0) {
         tc::tmem_alloc(tc::smem_u32(tslot), 512);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(s_mbar, 1);
-        tc::mbar_init(s_tbar, 1);
+        for (int i = 0; i < 11; ++i) tc::mbar_init(s_mbar + 8 * i, 1);
+        tc::mbar_arrive_expect_tx(s_xbar, 65 * 4);   // the peer's sums of chunk 0 (64 rows and a flag)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
+        flags[3] = 0;
+        pflag[0] = pflag[1] = 0;
     }
     if (tid < kDK) {
         gsv[tid] = p.gs ? p.gs[(size_t)h * kDK + tid] : 1.f;
         fprev[tid] = 1.f;
     }
     tc::fence_before_sync();
-    __syncthreads();
+    tc::cluster_sync();
     tc::fence_after_sync();
     const uint32_t tmem = *tslot;
-    uint32_t phase = 0, tphase = 0;
+    uint32_t phase = 0, rphase[2] = {0u, 0u};
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lanes
     const int row = 32 * (warp & 3) + lane;                         // accumulator row (M = 128)
-    const int colhalf = warp >> 2;                                  // 0: warps 0-3, 1: warps 4-7
+    const int colhalf = warp >> 2;                                  // 32-column half of this CTA's 64
     float range_max = 0.f;
 
-    // Wait for the MMAs committed so far; uniform abort on a timeout.
-    auto wait_mma = [&]() -> bool {
-        const bool ok = tc::mbar_wait(s_mbar, phase);
-        if (!ok) flags[0] = 1;
-        phase ^= 1u;
-        __syncthreads();
-        tc::fence_after_sync();
-        return flags[0] == 0;
-    };
+    if (warp < 8) {
+        // Wait for the MMAs committed so far; a timeout marks a local abort.
+        auto wait_mma = [&]() -> bool {
+            if (!tc::mbar_wait(s_mbar, phase)) flags[0] = 1;
+            phase ^= 1u;
+            main_sync();
+            tc::fence_after_sync();
+            return flags[0] == 0;
+        };
 
-    const size_t sbase = (size_t)head * kDK * kDV;
-    bool first = true;
-    bool prefetched = false;                      // the current window's record is already in flight
-    for (int w = 0; w < p.NW && flags[0] == 0; ++w) {
-    const int wend = min(T, kC * (w + 1));
-    // windows with precomputed chunk tiles (intra kernel) take the fast path;
-    // a flagged window (decay span too large for one 64-token chunk) is
-    // processed here in shorter chunks
-    const bool fast = p.ws != nullptr && p.wflags[(size_t)head * p.NW + w] == 0;
-    for (int t0 = kC * w; t0 < wend;) {
-        int n;
-        if (fast) {
-            const uint8_t *rec = p.ws + ((size_t)head * p.NW + w) * kWinBytes;
-            if (tid == 0 && !prefetched) {
-                tc::fence_proxy_async();
-                tc::mbar_arrive_expect_tx(s_tbar, kWinBytes - kWinPad);
-                tc::bulk_g2s(s_ap, rec + kWinAP, 128 * 256, s_tbar);
-                tc::bulk_g2s(s_bp, rec + kWinBP, 128 * 256, s_tbar);
-                tc::bulk_g2s(s_anab, rec + kWinANAB, 192 * 128, s_tbar);
-                tc::bulk_g2s(s_vh, rec + kWinVH, 64 * 2 * kDV, s_tbar);
-                tc::bulk_g2s(tc::smem_u32(ecv), rec + kWinVEC, 2 * 128 * 4, s_tbar);
+        const int NW = p.NW;
+        const size_t wbase = (size_t)head * NW;
+        auto win_fast = [&](int w) -> bool { return p.ws != nullptr && w < NW && p.wflags[wbase + w] == 0; };
+        auto issue_rec = [&](int w, int b) {         // thread 0: window w's record -> buffer b
+            const uint8_t *rec = p.ws + (wbase + w) * kWinBytes;
+            uint8_t *dst = sm + b * L::BUF;
+            const uint32_t bar = s_rbar + 8u * b;
+            tc::fence_proxy_async();
+            tc::mbar_arrive_expect_tx(bar, L::BUF);
+            tc::bulk_g2s(tc::smem_u32(dst + L::AP), rec + kWinAP, 128 * 256, bar);
+            tc::bulk_g2s(tc::smem_u32(dst + L::BP), rec + kWinBP, 128 * 256, bar);
+            tc::bulk_g2s(tc::smem_u32(dst + L::ANAB), rec + kWinANAB, 192 * 128, bar);
+            tc::bulk_g2s(tc::smem_u32(dst + L::VH), rec + kWinVH + crank * (64 * 128), 64 * 128, bar);
+            tc::bulk_g2s(tc::smem_u32(dst + L::EV), rec + kWinVEC, 2 * 128 * 4, bar);
+        };
+        static_assert(L::BUF == 2 * 128 * 256 + 192 * 128 + 64 * 128 + 1024, "record buffer = bytes of one record copy");
+
+        int loaded[2] = {-1, -1};                     // window whose record buffer b holds or receives
+        bool inflight[2] = {false, false};            // a copy into buffer b not yet waited for
+        for (int b = 0; b < 2; ++b)
+            if (win_fast(b)) {
+                if (tid == 0) issue_rec(b, b);
+                loaded[b] = b;
+                inflight[b] = true;
             }
-            // output gate of the window -> GS
-            {
-                const int tb = 8 * warp, c4 = 4 * lane;
+
+        const size_t sbase = (size_t)head * kDK * kDV;
+        bool first = true;
+        int chunk = 0;
+        uint32_t uses[2] = {0u, 0u};
+        for (int w = 0; w < NW && flags[0] == 0; ++w) {
+            const int B = w & 1;
+            uint8_t *buf = sm + B * L::BUF, *xbuf = sm + (B ^ 1) * L::BUF;
+            const uint32_t s_ap = tc::smem_u32(buf + L::AP), s_bp = tc::smem_u32(buf + L::BP);
+            const uint32_t s_anab = tc::smem_u32(buf + L::ANAB), s_vh = tc::smem_u32(buf + L::VH);
+            float *ecv = (float *)(buf + L::EV), *fcv = ecv + 128;
+            const int wend = min(T, kC * (w + 1));
+            const bool fast = loaded[B] == w;
+            // tile flag of window w + 2, loaded now and first compared once the window's
+            // products are done, so that its latency is hidden
+            const int wflag2 = (p.ws != nullptr && w + 2 < NW) ? __ldg(p.wflags + wbase + w + 2) : 1;
+            // an abort agreed by the readout warps becomes this group's abort at the barrier below
+            if (tid == 0 && flags[3] != 0) flags[0] = 1;
+            if (fast) {
+                if (!tc::mbar_wait(s_rbar + 8u * B, rphase[B])) flags[0] = 1;
+                rphase[B] ^= 1u;
+                inflight[B] = false;
+            } else if (inflight[B ^ 1]) {
+                // the other buffer is this window's scratch: a record arriving there
+                // lands first, and is copied again after the window
+                if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), rphase[B ^ 1])) flags[0] = 1;
+                rphase[B ^ 1] ^= 1u;
+                inflight[B ^ 1] = false;
+            }
+            main_sync();
+            for (int t0 = kC * w; t0 < wend && flags[0] == 0;) {
+                int n = wend - t0;
+                const uint32_t slot = (uint32_t)(chunk & 1);      // TMEM slot of this chunk's [R; O]
+                const uint32_t ro = kTmRO + (uint32_t)kDVC * slot;
+                ++chunk;
+                if (!fast && flags[0] == 0) do {
+                    // ---- A: loads, cumulative log-decay, span, chunk length.
+                    // Warp w owns tokens [8w, 8w+8); lane l owns key channels [4l, 4l+4)
+                    // and, for l < 16, value channels dv0 + [4l, 4l+4).
+                    float *wtot = (float *)(xbuf + L::WT), *probe = (float *)(xbuf + L::PR);
+                    float *spanred = (float *)(xbuf + L::XV), *diagq = spanred + 64, *diagb = spanred + 128;
+                    float *lw = (float *)(xbuf + L::LW), *yb = (float *)(xbuf + L::YB);
+                    const uint32_t s_ti = tc::smem_u32(xbuf + L::TI), s_mm = tc::smem_u32(xbuf + L::MM);
+                    const int tb = 8 * warp, c4 = 4 * lane;
+                    float la[8][4];
+                    uint2 kq[8][4];                           // [token][k, q, z, b]: 4 bf16 each
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int t = tb + u;
-                    const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + dv0 + c4;
-                    uint2 gg = make_uint2(0, 0);
-                    if (t0 + t < wend) gg = __ldg(reinterpret_cast<const uint2 *>(p.g + gv));
-                    *reinterpret_cast<uint2 *>(gsm + t * DVC + c4) = gg;
-                }
-            }
-            if (!tc::mbar_wait(s_tbar, tphase)) flags[0] = 1;
-            tphase ^= 1u;
-            __syncthreads();
-            if (flags[0]) break;
-            n = wend - t0;
-            prefetched = false;
-        } else {
-            // ---- A: loads, cumulative log-decay, span, chunk length.
-            // Warp w owns tokens [8w, 8w+8); lane l owns key channels [4l, 4l+4)
-            // and value channels [4l, 4l+4), so every load instruction reads whole
-            // 256-byte token rows.
-            const int tb = 8 * warp, c4 = 4 * lane;
-            float la[8][4];
-            uint2 kq[8][4];                           // [token][k, q, z, b]: 4 bf16 each
-    #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = tb + u;
-                const bool in = t0 + t < wend;
-                const size_t gk = (((size_t)bb * T + t0 + t) * H + h) * kDK + c4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (in) x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
-                la[u][0] = x.x; la[u][1] = x.y; la[u][2] = x.z; la[u][3] = x.w;
-                kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
-                kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-                kq[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-                kq[u][3] = in ? __ldg(reinterpret_cast<const uint2 *>(p.b + gk)) : make_uint2(0, 0);
-            }
-            // inclusive scan over tokens: within this warp's 8 tokens, then across warps
-    #pragma unroll
-            for (int u = 1; u < 8; ++u)
-    #pragma unroll
-                for (int c = 0; c < 4; ++c) la[u][c] += la[u - 1][c];
-            *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
-            __syncthreads();
-            {
-                float off[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int ww = 0; ww < warp; ++ww) {
-                    const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
-                    off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
-                }
-    #pragma unroll
-                for (int u = 0; u < 8; ++u)
-    #pragma unroll
-                    for (int c = 0; c < 4; ++c) la[u][c] += off[c];        // la now holds Lambda_t
-            }
-            // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j)
-    #pragma unroll
-            for (int j = 0; j < 7; ++j) {
-                const int pt = (1 << j) - 1;
-                if (pt >= tb && pt < tb + 8) {
-    #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (tb + u == pt)
-                            *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
-                                make_float4(la[u][0], la[u][1], la[u][2], la[u][3]);
-                }
-            }
-            __syncthreads();
-            {
-                // span of a chunk of 2^j tokens: max over this thread's 4 channels, then the CTA
-                const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
-                float sp[7];
-    #pragma unroll
-                for (int j = 0; j < 7; ++j) {
-                    const float4 lj = *reinterpret_cast<const float4 *>(probe + j * kDK + c4);
-                    float m = fmaxf(fmaxf(l0.x - lj.x, l0.y - lj.y), fmaxf(l0.z - lj.z, l0.w - lj.w));
-    #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    sp[j] = m;
-                }
-                if (lane == 0)
-    #pragma unroll
-                    for (int j = 0; j < 7; ++j) spanred[warp * 8 + j] = sp[j];
-            }
-            __syncthreads();
-            if (tid == 0) {
-                int nj = 0;
-                for (int j = 6; j >= 0; --j) {
-                    float m = 0.f;
-                    for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, spanred[ww * 8 + j]);
-                    if (m <= kSpanMax) { nj = j; break; }
-                }
-                flags[1] = min(1 << nj, wend - t0);
-                flags[2] = nj;
-            }
-            // value-side loads (their latency overlaps the operand computation)
-            uint2 vw[8][3];                           // [token][v, w, g]
-    #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = tb + u;
-                const bool in = t0 + t < wend;
-                const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + dv0 + c4;
-                vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
-                vw[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.g + gv)) : make_uint2(0, 0);
-            }
-            __syncthreads();
-            n = flags[1];
-
-            // ---- B: operand tiles (fp16, swizzled), pivot vectors, exact diagonals
-            {
-                // Lambda_{n-1} is the probe of the chosen power-of-two chunk: past the
-                // end of the sequence the log-decay is zero-padded, so a shorter tail
-                // has the same cumulative value there.
-                const int jn = flags[2];
-                const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
-                const float4 ln4 = *reinterpret_cast<const float4 *>(probe + jn * kDK + c4);
-                const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
-                const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
-                float cpiv[4], gq[4];
-    #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    cpiv[c] = 0.5f * (l0v[c] + lnv[c]);
-                    gq[c] = gsv[c4 + c];
-                    if (warp == 0) {
-                        ecv[c4 + c] = __expf(cpiv[c]);
-                        fcv[c4 + c] = __expf(lnv[c] - cpiv[c]);
-                    }
-                }
-    #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int t = tb + u;
-                    const bool live = t < n;
-                    float kk[4], qq[4], zz[4], bv[4];
-                    {
-                        const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][0]);
-                        const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][1]);
-                        const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][2]);
-                        const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][3]);
-    #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            float2 f;
-                            f = __bfloat1622float2(hk[e]); kk[2 * e] = f.x; kk[2 * e + 1] = f.y;
-                            f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
-                            f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
-                            f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
-                        }
-                    }
-                    float kp[4], kc[4], khc[4], qp[4];
-                    float dq = 0.f, db = 0.f;
-    #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float lam = live ? la[u][c] : lnv[c];     // identity padding past n
-                        const float d = lam - cpiv[c];
-                        const float ep = __expf(d), em = __expf(-d);
-                        const float kv = live ? kk[c] : 0.f;
-                        const float qt = live ? qq[c] * gq[c] * (2.f / (1.f + __expf(-zz[c]))) : 0.f;
-                        const float kh = bv[c] * kv;
-                        dq += qt * kv;
-                        db += qt * kh;
-                        kp[c] = kv * ep;
-                        kc[c] = kv * em;
-                        khc[c] = kh * em;
-                        qp[c] = qt * ep;
-                    }
-                    range_max = fmaxf(range_max, fmaxf(fmaxf(maxabs(kp, 4), maxabs(kc, 4)),
-                                                       fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
-                    // the diagonal of Aq / Bq carries no decay: it is summed exactly in
-                    // fp32 (a readout whose q~.k nearly cancels, e.g. the first token of a
-                    // sequence, is then free of fp16 operand rounding)
-    #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        dq += __shfl_xor_sync(0xffffffffu, dq, o);
-                        db += __shfl_xor_sync(0xffffffffu, db, o);
-                    }
-                    if (lane == 0) {
-                        diagq[t] = dq;
-                        diagb[t] = db;
-                    }
-                    const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
-                    *(uint2 *)(sm + L::AP + off_t) = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
-                    *(uint2 *)(sm + L::AP + off_b) = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
-                    *(uint2 *)(sm + L::BP + off_t) = make_uint2(tc::pack_half2(kc[0], kc[1]), tc::pack_half2(kc[2], kc[3]));
-                    *(uint2 *)(sm + L::BP + off_b) =
-                        make_uint2(tc::pack_half2(khc[0], khc[1]), tc::pack_half2(khc[2], khc[3]));
-                }
-                if (c4 < DVC) {
-    #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int t = tb + u;
-                        const bool live = t < n;
-                        const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
-                        const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
-                        float vh[4];
-    #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const float2 fv = __bfloat1622float2(hv[e]), fw = __bfloat1622float2(hw[e]);
-                            vh[2 * e] = live ? fv.x * fw.x : 0.f;
-                            vh[2 * e + 1] = live ? fv.y * fw.y : 0.f;
+                        const bool in = t0 + t < wend;
+                        const size_t gk = (((size_t)bb * T + t0 + t) * H + h) * kDK + c4;
+                        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (in) x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                        la[u][0] = x.x; la[u][1] = x.y; la[u][2] = x.z; la[u][3] = x.w;
+                        kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
+                        kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
+                        kq[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+                        kq[u][3] = in ? __ldg(reinterpret_cast<const uint2 *>(p.b + gk)) : make_uint2(0, 0);
+                    }
+                    // inclusive scan over tokens: within this warp's 8 tokens, then across warps
+#pragma unroll
+                    for (int u = 1; u < 8; ++u)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) la[u][c] += la[u - 1][c];
+                    *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
+                    main_sync();
+                    {
+                        float off[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int ww = 0; ww < warp; ++ww) {
+                            const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
+                            off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
                         }
-                        *(uint2 *)(sm + L::VH + tc::tile_off(64, t, c4)) =
-                            make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
-                        *reinterpret_cast<uint2 *>(gsm + t * DVC + c4) = vw[u][2];
-                    }
-                }
-            }
-            tc::fence_proxy_async();
-            __syncthreads();
-
-            // ---- C: decay-relative products P = [Kp; Qp] [Kc; K^c]^T
-            if (tid == 0) {
-                tc::fence_after_sync();
-                const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
-                for (int ks = 0; ks < kDK / 16; ++ks)
-                    tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id,
-                                ks > 0);
-                tc::mma_commit(s_mbar);
-            }
-            if (!wait_mma()) break;
-
-            // ---- D: masks; M -> MM, L -> fp32, Aq/Bq -> ANAB
-            {
-                // rows 0-63: warps 0,1 (M, cols 0-63) and warps 4,5 (L, cols 64-127)
-                // rows 64-127: warps 2,3 (Aq) and warps 6,7 (Bq)
-                const int t = row & 63;
-                const bool upper = row < 64;
-                float v[2][32];
-                tc::tmem_ld32x2(tmem + lane_base + kTmP + 64 * colhalf, tmem + lane_base + kTmP + 64 * colhalf + 32,
-                                v[0], v[1]);
-    #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = 32 * hf + i;
-                        const bool keep = upper ? (s < t) : (s <= t);
-                        if (!keep) v[hf][i] = 0.f;
-                        if (!upper && s == t) v[hf][i] = colhalf == 0 ? diagq[t] : diagb[t];
-                    }
-                    if (upper && colhalf == 1) {
-                        float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
-    #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(v[hf][4 * q], v[hf][4 * q + 1], v[hf][4 * q + 2], v[hf][4 * q + 3]);
-                    } else {
-                        uint8_t *tile = upper ? sm + L::MM : sm + L::ANAB;
-                        const int R = upper ? 64 : 192;
-                        const int r = upper ? t : (colhalf == 0 ? 64 + t : 128 + t);
-                        store_row32(tile, R, r, 32 * hf, v[hf]);
-                    }
-                }
-            }
-            tc::fence_before_sync();
-            __syncthreads();
-
-            // ---- E: T^-1 = (I + L)^-1 in place, divide and conquer (fp32)
-            {
-                // leaves of 8: forward substitution per column, in registers
-                if (tid < 64) {
-                    const int o = 8 * (tid >> 3), j = tid & 7;
-                    float Lr[8][8];
-    #pragma unroll
-                    for (int i = 1; i < 8; ++i)
-    #pragma unroll
-                        for (int s = 0; s < i; ++s) Lr[i][s] = lw[(o + i) * kLW + o + s];
-                    float x[8];
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i) x[i] = (i == j) ? 1.f : 0.f;
-    #pragma unroll
-                    for (int i = 1; i < 8; ++i) {
-                        float acc = 0.f;
-    #pragma unroll
-                        for (int s = 0; s < i; ++s) acc += Lr[i][s] * x[s];
-                        if (i > j) x[i] = -acc;
-                    }
-                    __syncwarp();
-                    asm volatile("bar.sync 1, 64;" ::: "memory");     // the 64 leaf threads only
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (i >= j) lw[(o + i) * kLW + o + j] = x[i];
-                }
-                __syncthreads();
-                // merges: [[A, 0], [C, D]]^-1 = [[A^-1, 0], [-D^-1 C A^-1, D^-1]],
-                // four output columns per task; the upper triangles are zero, so the
-                // sums run over whole blocks without masks
-                merge_level<8>(lw, yb, tid);
-                merge_level<16>(lw, yb, tid);
-                merge_level<32>(lw, yb, tid);
-                // T^-1 -> fp16 tile (row t, column s; the upper part of lw is zero)
-                for (int u = tid; u < 64 * 8; u += kThreads) {
-                    const int t = u >> 3, g8 = u & 7;
-                    const float4 a = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8 + 4);
-                    const float f[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-                    *(uint4 *)(sm + L::TI + tc::tile_chunk_off(64, t, g8)) = pack8(f);
-                }
-            }
-            tc::fence_proxy_async();
-            __syncthreads();
-
-            // ---- F: W' = T^-1 Kp, N = T^-1 M
-            if (tid == 0) {
-                tc::fence_after_sync();
-                const uint32_t idw = tc::idesc_f16(64, 128, false, true, false);
-                const uint32_t idn = tc::idesc_f16(64, 64, false, true, false);
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    tc::mma_f16(tmem + kTmW, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_ap, 128, 0, ks), idw,
-                                ks > 0);
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    tc::mma_f16(tmem + kTmN, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_mm, 64, 0, ks), idn,
-                                ks > 0);
-                tc::mma_commit(s_mbar);
-            }
-            if (!wait_mma()) break;
-
-            // ---- G: W' -> rows 0-63 of AP (over Kp), N -> rows 0-63 of ANAB.
-            // M = 64 accumulators sit in lanes 0-15 of each 32-lane group.
-            {
-                const int t = 16 * (warp & 3) + lane;
-                const bool valid = lane < 16;
-                float v[2][32];
-                // warps 0-3: W' columns 0-63; warps 4-7: W' columns 64-127
-                tc::tmem_ld32x2(tmem + lane_base + kTmW + 64 * colhalf, tmem + lane_base + kTmW + 64 * colhalf + 32, v[0],
-                                v[1]);
-                if (valid) {
-    #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        range_max = fmaxf(range_max, maxabs(v[hf], 32));
-                        store_row32(sm + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
-                    }
-                }
-                // warps 0-3: N columns 0-31; warps 4-7: N columns 32-63
-                float nv[32];
-                tc::tmem_ld32(tmem + lane_base + kTmN + 32 * colhalf, nv);
-                if (valid) {
-                    range_max = fmaxf(range_max, maxabs(nv, 32));
-                    store_row32(sm + L::ANAB, 192, t, 32 * colhalf, nv);
-                }
-            }
-
-        }
-        // ---- H: state operand S_c = Diag(e^c) S, X <- S_c (fp32, TMEM)
-        {
-            const int i = row;                                   // key channel
-            const float scale = ecv[i] * fprev[i];
-            for (int cblk = 0; cblk < DVC / 64; ++cblk) {
-                const int col = (DVC / 2) * colhalf + 32 * cblk;
-                float v[32];
-                if (first) {
-                    if (p.S_in) {
-                        const float4 *src = reinterpret_cast<const float4 *>(p.S_in + sbase + (size_t)i * kDV + dv0 + col);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 x4 = __ldg(src + q);
-                            v[4 * q] = x4.x; v[4 * q + 1] = x4.y; v[4 * q + 2] = x4.z; v[4 * q + 3] = x4.w;
+                        for (int u = 0; u < 8; ++u)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) la[u][c] += off[c];        // la now holds Lambda_t
+                    }
+                    // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j)
+#pragma unroll
+                    for (int j = 0; j < 7; ++j) {
+                        const int pt = (1 << j) - 1;
+                        if (pt >= tb && pt < tb + 8) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                if (tb + u == pt)
+                                    *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
+                                        make_float4(la[u][0], la[u][1], la[u][2], la[u][3]);
                         }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q] = 0.f;
                     }
-                } else {
-                    tc::tmem_ld32(tmem + lane_base + kTmX + col, v);
-                }
+                    main_sync();
+                    {
+                        // span of a chunk of 2^j tokens: max over this thread's 4 channels, then the CTA
+                        const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
+                        float sp[7];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] *= scale;
-                tc::tmem_st32(tmem + lane_base + kTmX + col, v);
-                range_max = fmaxf(range_max, maxabs(v, 32));
-                store_row32(sm + L::SC, 128, i, col, v);
-            }
-        }
-        first = false;
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // ---- I: [R; O] = [W'; Qp] S_c + [N; Aq] V^ ;  X += Kc^T V^
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t id1 = tc::idesc_f16(128, DVC, false, true, false);
-            for (int ks = 0; ks < kDK / 16; ++ks)
-                tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_mnmajor(s_sc, 128, 0, ks), id1,
-                            ks > 0);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_anab, 192, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks), id1,
-                            true);
-            const uint32_t id2 = tc::idesc_f16(128, DVC, true, true, false);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks), id2,
-                            true);
-            tc::mma_commit(s_mbar);
-        }
-        if (!wait_mma()) break;
-
-        // ---- J: R (rows 0-63) -> fp16 tile
-        if (row < 64) {
-            float v[2][32];
-            tc::tmem_ld32x2(tmem + lane_base + kTmP + (DVC / 2) * colhalf,
-                            tmem + lane_base + kTmP + (DVC / 2) * colhalf + 32, v[0], v[1]);
+                        for (int j = 0; j < 7; ++j) {
+                            const float4 lj = *reinterpret_cast<const float4 *>(probe + j * kDK + c4);
+                            float m = fmaxf(fmaxf(l0.x - lj.x, l0.y - lj.y), fmaxf(l0.z - lj.z, l0.w - lj.w));
 #pragma unroll
-            for (int hf = 0; hf < DVC / 64; ++hf) {
-                range_max = fmaxf(range_max, maxabs(v[hf], 32));
-                store_row32(sm + L::RR, 64, row, (DVC / 2) * colhalf + 32 * hf, v[hf]);
-            }
-        }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
+                            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                            sp[j] = m;
+                        }
+                        if (lane == 0)
+#pragma unroll
+                            for (int j = 0; j < 7; ++j) spanred[warp * 8 + j] = sp[j];
+                    }
+                    main_sync();
+                    if (tid == 0) {
+                        int nj = 0;
+                        for (int j = 6; j >= 0; --j) {
+                            float m = 0.f;
+                            for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, spanred[ww * 8 + j]);
+                            if (m <= kSpanMax) { nj = j; break; }
+                        }
+                        flags[1] = min(1 << nj, wend - t0);
+                        flags[2] = nj;
+                    }
+                    // value-side loads (their latency overlaps the operand computation)
+                    const bool vlane = c4 < kDVC;
+                    uint2 vw[8][2];                           // [token][v, w]
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int t = tb + u;
+                        const bool in = t0 + t < wend && vlane;
+                        const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + dv0 + c4;
+                        vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+                        vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
+                    }
+                    main_sync();
+                    n = flags[1];
 
-        // ---- K: O -= Bq R (rows 64-127; rows 0-63 receive -Aq R, unused);  X -= K^c^T R
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t id1 = tc::idesc_f16(128, DVC, false, true, true);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_anab, 192, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks), id1,
-                            true);
-            const uint32_t id2 = tc::idesc_f16(128, DVC, true, true, true);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks), id2,
-                            true);
-            tc::mma_commit(s_mbar);
-        }
-        if (!wait_mma()) break;
-        // the chunk's tiles are free: keep its decay factor, then start the
-        // bulk copy of the next window's record so it overlaps the epilogue
-        if (tid < kDK) fprev[tid] = fcv[tid];
-        {
-            const bool next_fast = t0 + n == wend && w + 1 < p.NW && p.ws != nullptr &&
-                                   p.wflags[(size_t)head * p.NW + w + 1] == 0;
-            __syncthreads();
-            if (next_fast) {
-                if (tid == 0) {
-                    const uint8_t *nrec = p.ws + ((size_t)head * p.NW + w + 1) * kWinBytes;
+                    // ---- B: operand tiles (fp16, swizzled), pivot vectors, exact diagonals
+                    {
+                        // Lambda_{n-1} is the probe of the chosen power-of-two chunk: past the
+                        // end of the sequence the log-decay is zero-padded, so a shorter tail
+                        // has the same cumulative value there.
+                        const int jn = flags[2];
+                        const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
+                        const float4 ln4 = *reinterpret_cast<const float4 *>(probe + jn * kDK + c4);
+                        const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
+                        const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
+                        float cpiv[4], gq[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            cpiv[c] = 0.5f * (l0v[c] + lnv[c]);
+                            gq[c] = gsv[c4 + c];
+                            if (warp == 0) {
+                                ecv[c4 + c] = __expf(cpiv[c]);
+                                fcv[c4 + c] = __expf(lnv[c] - cpiv[c]);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int t = tb + u;
+                            const bool live = t < n;
+                            float kk[4], qq[4], zz[4], bv[4];
+                            {
+                                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][0]);
+                                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][1]);
+                                const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][2]);
+                                const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][3]);
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    float2 f;
+                                    f = __bfloat1622float2(hk[e]); kk[2 * e] = f.x; kk[2 * e + 1] = f.y;
+                                    f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
+                                    f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
+                                    f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
+                                }
+                            }
+                            float kp[4], kc[4], khc[4], qp[4];
+                            float dq = 0.f, db = 0.f;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const float lam = live ? la[u][c] : lnv[c];     // identity padding past n
+                                const float d = lam - cpiv[c];
+                                const float ep = __expf(d), em = __expf(-d);
+                                const float kv = live ? kk[c] : 0.f;
+                                const float qt = live ? qq[c] * gq[c] * (2.f / (1.f + __expf(-zz[c]))) : 0.f;
+                                const float kh = bv[c] * kv;
+                                dq += qt * kv;
+                                db += qt * kh;
+                                kp[c] = kv * ep;
+                                kc[c] = kv * em;
+                                khc[c] = kh * em;
+                                qp[c] = qt * ep;
+                            }
+                            range_max = fmaxf(range_max, fmaxf(fmaxf(maxabs(kp, 4), maxabs(kc, 4)),
+                                                               fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
+                            // the diagonal of Aq / Bq carries no decay: it is summed exactly in
+                            // fp32 (a readout whose q~.k nearly cancels, e.g. the first token of a
+                            // sequence, is then free of fp16 operand rounding)
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) {
+                                dq += __shfl_xor_sync(0xffffffffu, dq, o);
+                                db += __shfl_xor_sync(0xffffffffu, db, o);
+                            }
+                            if (lane == 0) {
+                                diagq[t] = dq;
+                                diagb[t] = db;
+                            }
+                            const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
+                            *(uint2 *)(buf + L::AP + off_t) = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
+                            *(uint2 *)(buf + L::AP + off_b) = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
+                            *(uint2 *)(buf + L::BP + off_t) = make_uint2(tc::pack_half2(kc[0], kc[1]), tc::pack_half2(kc[2], kc[3]));
+                            *(uint2 *)(buf + L::BP + off_b) =
+                                make_uint2(tc::pack_half2(khc[0], khc[1]), tc::pack_half2(khc[2], khc[3]));
+                        }
+                        if (vlane) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int t = tb + u;
+                                const bool live = t < n;
+                                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
+                                const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
+                                float vh[4];
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const float2 fv = __bfloat1622float2(hv[e]), fw = __bfloat1622float2(hw[e]);
+                                    vh[2 * e] = live ? fv.x * fw.x : 0.f;
+                                    vh[2 * e + 1] = live ? fv.y * fw.y : 0.f;
+                                }
+                                *(uint2 *)(buf + L::VH + tc::tile_off(64, t, c4)) =
+                                    make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
+                            }
+                        }
+                    }
                     tc::fence_proxy_async();
-                    tc::mbar_arrive_expect_tx(s_tbar, kWinBytes - kWinPad);
-                    tc::bulk_g2s(s_ap, nrec + kWinAP, 128 * 256, s_tbar);
-                    tc::bulk_g2s(s_bp, nrec + kWinBP, 128 * 256, s_tbar);
-                    tc::bulk_g2s(s_anab, nrec + kWinANAB, 192 * 128, s_tbar);
-                    tc::bulk_g2s(s_vh, nrec + kWinVH, 64 * 2 * kDV, s_tbar);
-                    tc::bulk_g2s(tc::smem_u32(ecv), nrec + kWinVEC, 2 * 128 * 4, s_tbar);
+                    main_sync();
+
+                    // ---- C: decay-relative products P = [Kp; Qp] [Kc; K^c]^T
+                    if (tid == 0) {
+                        tc::fence_after_sync();
+                        const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
+                        for (int ks = 0; ks < kDK / 16; ++ks)
+                            tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id,
+                                        ks > 0);
+                        tc::mma_commit(s_mbar);
+                    }
+                    if (!wait_mma()) break;
+
+                    // ---- D: masks; M -> MM, L -> fp32, Aq/Bq -> ANAB
+                    {
+                        // rows 0-63: warps 0,1 (M, cols 0-63) and warps 4,5 (L, cols 64-127)
+                        // rows 64-127: warps 2,3 (Aq) and warps 6,7 (Bq)
+                        const int t = row & 63;
+                        const bool upper = row < 64;
+                        float v[2][32];
+                        tc::tmem_ld32x2(tmem + lane_base + kTmP + 64 * colhalf, tmem + lane_base + kTmP + 64 * colhalf + 32,
+                                        v[0], v[1]);
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const int s = 32 * hf + i;
+                                const bool keep = upper ? (s < t) : (s <= t);
+                                if (!keep) v[hf][i] = 0.f;
+                                if (!upper && s == t) v[hf][i] = colhalf == 0 ? diagq[t] : diagb[t];
+                            }
+                            if (upper && colhalf == 1) {
+                                float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    dst[q] = make_float4(v[hf][4 * q], v[hf][4 * q + 1], v[hf][4 * q + 2], v[hf][4 * q + 3]);
+                            } else {
+                                uint8_t *tile = upper ? xbuf + L::MM : buf + L::ANAB;
+                                const int R = upper ? 64 : 192;
+                                const int r = upper ? t : (colhalf == 0 ? 64 + t : 128 + t);
+                                store_row32(tile, R, r, 32 * hf, v[hf]);
+                            }
+                        }
+                    }
+                    tc::fence_before_sync();
+                    main_sync();
+
+                    // ---- E: T^-1 = (I + L)^-1 in place, divide and conquer (fp32)
+                    {
+                        // leaves of 8: forward substitution per column, in registers
+                        if (tid < 64) {
+                            const int o = 8 * (tid >> 3), j = tid & 7;
+                            float Lr[8][8];
+#pragma unroll
+                            for (int i = 1; i < 8; ++i)
+#pragma unroll
+                                for (int s = 0; s < i; ++s) Lr[i][s] = lw[(o + i) * kLW + o + s];
+                            float x[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) x[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                            for (int i = 1; i < 8; ++i) {
+                                float acc = 0.f;
+#pragma unroll
+                                for (int s = 0; s < i; ++s) acc += Lr[i][s] * x[s];
+                                if (i > j) x[i] = -acc;
+                            }
+                            __syncwarp();
+                            asm volatile("bar.sync 2, 64;" ::: "memory");     // the 64 leaf threads only
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                if (i >= j) lw[(o + i) * kLW + o + j] = x[i];
+                        }
+                        main_sync();
+                        // merges: [[A, 0], [C, D]]^-1 = [[A^-1, 0], [-D^-1 C A^-1, D^-1]],
+                        // four output columns per task; the upper triangles are zero, so the
+                        // sums run over whole blocks without masks
+                        merge_level<8>(lw, yb, tid);
+                        merge_level<16>(lw, yb, tid);
+                        merge_level<32>(lw, yb, tid);
+                        // T^-1 -> fp16 tile (row t, column s; the upper part of lw is zero)
+                        for (int u = tid; u < 64 * 8; u += kThreads) {
+                            const int t = u >> 3, g8 = u & 7;
+                            const float4 a = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8);
+                            const float4 b4 = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8 + 4);
+                            const float f[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
+                            *(uint4 *)(xbuf + L::TI + tc::tile_chunk_off(64, t, g8)) = pack8(f);
+                        }
+                    }
+                    tc::fence_proxy_async();
+                    main_sync();
+
+                    // ---- F: W' = T^-1 Kp, N = T^-1 M
+                    if (tid == 0) {
+                        tc::fence_after_sync();
+                        const uint32_t idw = tc::idesc_f16(64, 128, false, true, false);
+                        const uint32_t idn = tc::idesc_f16(64, 64, false, true, false);
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::mma_f16(tmem + kTmW, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_ap, 128, 0, ks), idw,
+                                        ks > 0);
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::mma_f16(tmem + kTmN, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_mm, 64, 0, ks), idn,
+                                        ks > 0);
+                        tc::mma_commit(s_mbar);
+                    }
+                    if (!wait_mma()) break;
+
+                    // ---- G: W' -> rows 0-63 of AP (over Kp), N -> rows 0-63 of ANAB.
+                    // M = 64 accumulators sit in lanes 0-15 of each 32-lane group.
+                    {
+                        const int t = 16 * (warp & 3) + lane;
+                        const bool valid = lane < 16;
+                        float v[2][32];
+                        // warps 0-3: W' columns 0-63; warps 4-7: W' columns 64-127
+                        tc::tmem_ld32x2(tmem + lane_base + kTmW + 64 * colhalf, tmem + lane_base + kTmW + 64 * colhalf + 32,
+                                        v[0], v[1]);
+                        if (valid) {
+#pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+                                range_max = fmaxf(range_max, maxabs(v[hf], 32));
+                                store_row32(buf + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
+                            }
+                        }
+                        // warps 0-3: N columns 0-31; warps 4-7: N columns 32-63
+                        float nv[32];
+                        tc::tmem_ld32(tmem + lane_base + kTmN + 32 * colhalf, nv);
+                        if (valid) {
+                            range_max = fmaxf(range_max, maxabs(nv, 32));
+                            store_row32(buf + L::ANAB, 192, t, 32 * colhalf, nv);
+                        }
+                    }
+                } while (false);
+
+                if (flags[0] == 0) {
+                    // ---- H: state operand S_c = Diag(e^c) S, X <- S_c (fp32, TMEM)
+                    {
+                        const int i = row;                                   // key channel
+                        const float scale = ecv[i] * fprev[i];
+                        const int col = 32 * colhalf;
+                        float v[32];
+                        if (first) {
+                            if (p.S_in) {
+                                const float4 *src =
+                                    reinterpret_cast<const float4 *>(p.S_in + sbase + (size_t)i * kDV + dv0 + col);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const float4 x4 = __ldg(src + q);
+                                    v[4 * q] = x4.x; v[4 * q + 1] = x4.y; v[4 * q + 2] = x4.z; v[4 * q + 3] = x4.w;
+                                }
+                            } else {
+#pragma unroll
+                                for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                            }
+                        } else {
+                            tc::tmem_ld32(tmem + lane_base + kTmX + col, v);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) v[q] *= scale;
+                        tc::tmem_st32(tmem + lane_base + kTmX + col, v);
+                        range_max = fmaxf(range_max, maxabs(v, 32));
+                        store_row32(sm + L::SC, 128, i, col, v);
+                    }
+                    first = false;
+                    tc::fence_proxy_async();
+                    tc::fence_before_sync();
+                    main_sync();
+
+                    // ---- I: [R; O] = [W'; Qp] S_c + [N; Aq] V^ ;  X += Kc^T V^
+                    if (tid == 0) {
+                        // the slot's previous O has been read out of TMEM (and its chunk info)
+                        if (uses[slot] > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u)) flags[0] = 1;
+                        // the readout warps learn the chunk's tokens now (to fetch the gate early)
+                        info[4 * slot] = t0;
+                        info[4 * slot + 1] = n;
+                        info[4 * slot + 2] = 0;
+                        tc::mbar_arrive_local(s_ibar + 8u * slot);
+                        tc::fence_after_sync();
+                        const uint32_t id1 = tc::idesc_f16(128, kDVC, false, true, false);
+                        if (flags[0] == 0) {
+                            for (int ks = 0; ks < kDK / 16; ++ks)
+                                tc::mma_f16(tmem + ro, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_mnmajor(s_sc, 128, 0, ks),
+                                            id1, ks > 0);
+                            for (int ks = 0; ks < kC / 16; ++ks)
+                                tc::mma_f16(tmem + ro, tc::desc_kmajor(s_anab, 192, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks),
+                                            id1, true);
+                        }
+                        tc::mma_commit(s_mbar);                   // [R; O]: R is read out next
+                        // the state's V^ term runs on the tensor core while R is read out
+                        // (the next commit covers it)
+                        const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, false);
+                        if (flags[0] == 0)
+                            for (int ks = 0; ks < kC / 16; ++ks)
+                                tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks),
+                                            id2, true);
+                    }
                 }
-                prefetched = true;
+                if (flags[0] == 0 && wait_mma()) {
+                    // ---- J: R (rows 0-63) -> fp16 tile
+                    if (row < 64) {
+                        float v[32];
+                        tc::tmem_ld32(tmem + lane_base + ro + 32 * colhalf, v);
+                        range_max = fmaxf(range_max, maxabs(v, 32));
+                        store_row32(sm + L::RR, 64, row, 32 * colhalf, v);
+                    }
+                    tc::fence_proxy_async();
+                    tc::fence_before_sync();
+                    main_sync();
+
+                    // ---- K: O -= Bq R (rows 64-127; rows 0-63 receive -Aq R, unused);  X -= K^c^T R
+                    if (tid == 0) {
+                        tc::fence_after_sync();
+                        const uint32_t id1 = tc::idesc_f16(128, kDVC, false, true, true);
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::mma_f16(tmem + ro, tc::desc_kmajor(s_anab, 192, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks),
+                                        id1, true);
+                        const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, true);
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks),
+                                        id2, true);
+                        tc::mma_commit(s_mbar);
+                        tc::mma_commit(s_obar + 8u * slot);      // O of this chunk is final
+                    }
+                    if (wait_mma()) {
+                        // the chunk's tiles are free: keep its decay factor; once the window's
+                        // last chunk is done, its buffer takes the record of window w + 2
+                        if (tid < kDK) fprev[tid] = fcv[tid];
+                        main_sync();
+                        if (t0 + n == wend) {
+                            if (wflag2 == 0) {
+                                if (tid == 0) issue_rec(w + 2, B);
+                                loaded[B] = w + 2;
+                                inflight[B] = true;
+                            } else {
+                                loaded[B] = -1;
+                            }
+                        }
+                    }
+                }
+
+                tc::fence_before_sync();
+                main_sync();
+                tc::fence_after_sync();
+                ++uses[slot];
+                t0 += n;
+            }
+            // after a window processed in shorter chunks: the record of window w + 1
+            // (its scratch buffer) is copied again, and this buffer takes window w + 2
+            if (!fast && flags[0] == 0) {
+                if (loaded[B ^ 1] == w + 1) {
+                    if (tid == 0) issue_rec(w + 1, B ^ 1);
+                    inflight[B ^ 1] = true;
+                }
             }
         }
 
-        // ---- L: O (rows 64-127) -> RMSNorm over the head's d_v, gate, store
-        {
-            const bool orow = row >= 64;
-            const int t = row - 64;
+        // no more chunks: tell the readout warps
+        if (tid == 0) {
+            const uint32_t slot = (uint32_t)(chunk & 1);
+            if (uses[slot] > 0) tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u);
+            info[4 * slot + 2] = 1;
+            tc::mbar_arrive_local(s_ibar + 8u * slot);
+        }
+        // copies still in flight (the loop ended early) complete before exit
+        for (int b = 0; b < 2; ++b)
+            if (inflight[b]) tc::mbar_wait(s_rbar + 8u * b, rphase[b]);
+
+        // ---- S_out = Diag(fprev) X
+        if (flags[0] == 0 && p.S_out && T > 0) {
+            const int i = row;
+            const int col = 32 * colhalf;
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + kTmX + col, v);
+            float4 *dst = reinterpret_cast<float4 *>(p.S_out + sbase + (size_t)i * kDV + dv0 + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(v[4 * q] * fprev[i], v[4 * q + 1] * fprev[i], v[4 * q + 2] * fprev[i],
+                                     v[4 * q + 3] * fprev[i]);
+        }
+    } else if (warp >= 10) {
+        // ---- readout warps: O (TMEM lanes 64-127) -> RMS norm over d_v (both
+        // CTAs' columns, exchanged through distributed shared memory), gate, store
+        const int et = tid - 320;                    // token row of the chunk
+        for (int c = 0;; ++c) {
+            const uint32_t slot = (uint32_t)(c & 1), ph = (uint32_t)(c >> 1) & 1u;
+            // one thread waits, the barrier hands its view (and the chunk info) to the rest
+            if (et == 0 && !tc::mbar_wait(s_ibar + 8u * slot, ph)) flags[3] = 1;
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            if (flags[3] != 0) break;
+            // every row is done with the previous chunk's exchange slot: it now
+            // expects the peer's sums of chunk c + 1
+            if (et == 0) tc::mbar_arrive_expect_tx(s_xbar + 8u * (slot ^ 1u), 65 * 4);
+            const int t0 = info[4 * slot], n = info[4 * slot + 1];
+            if (info[4 * slot + 2] != 0) break;      // no more chunks
+            // the gate of this row, fetched while the chunk's products run
+            const bool live = et < n;
+            const size_t gi = (((size_t)bb * T + t0 + et) * H + h) * kDV + dv0;
+            uint4 gq[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                gq[q] = live ? __ldg(reinterpret_cast<const uint4 *>(p.g + gi) + q) : make_uint4(0, 0, 0, 0);
+            bool ok = true;
+            if (et == 0) ok = tc::mbar_wait(s_obar + 8u * slot, ph);
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            tc::fence_after_sync();
             float ov[2][32];
+            const uint32_t ro = kTmRO + (uint32_t)kDVC * slot;
+            tc::tmem_ld32x2(tmem + lane_base + ro, tmem + lane_base + ro + 32, ov[0], ov[1]);
+            tc::fence_before_sync();
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            if (et == 0) tc::mbar_arrive_local(s_fbar + 8u * slot);   // the slot may take a new chunk
             float ss = 0.f;
-            if (orow) {
-                tc::tmem_ld32x2(tmem + lane_base + kTmP + (DVC / 2) * colhalf,
-                                tmem + lane_base + kTmP + (DVC / 2) * colhalf + 32, ov[0], ov[1]);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) ss += ov[hf][q] * ov[hf][q];
-                part[t * 2 + colhalf] = ss;
+                for (int q = 0; q < 32; ++q) ss += ov[hf][q] * ov[hf][q];
+            // exchange: this row's sum (and the abort flag) into the peer's slot as
+            // asynchronous stores counted on the peer's barrier
+            tc::st_async_f32(r_peer + slot * 256u + 4u * et, ss, r_xbar + 8u * slot);
+            if (et == 0) tc::st_async_s32(r_pflag + 4u * slot, (ok && flags[0] == 0) ? 0 : 1, r_xbar + 8u * slot);
+            if (et == 0) {
+                const bool got = tc::mbar_wait_cluster(s_xbar + 8u * slot, ph);
+                if (!got || pflag[slot] != 0 || !ok) flags[3] = 1;
             }
-            __syncthreads();
-            if (orow && t < n) {
-                const float tot = part[t * 2] + part[t * 2 + 1];
-                const float inv = rsqrtf(tot / kDV + p.eps);
-                const int c0 = (DVC / 2) * colhalf;
-                const size_t gi = (((size_t)bb * T + t0 + t) * H + h) * kDV + dv0 + c0;
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            if (flags[3] != 0) break;
+            if (live) {
+                const float inv = rsqrtf((ss + peer[slot * 64 + et]) / kDV + p.eps);
 #pragma unroll
-                for (int q8 = 0; q8 < DVC / 16; ++q8) {
+                for (int q8 = 0; q8 < 8; ++q8) {
                     float gg[8], yy[8];
-                    bf16x8_to_f(*reinterpret_cast<const uint4 *>(gsm + t * DVC + c0 + 8 * q8), gg);
+                    bf16x8_to_f(gq[q8], gg);
                     const float *o8 = &ov[q8 >> 2][8 * (q8 & 3)];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) yy[e] = gg[e] * o8[e] * inv;
@@ -782,35 +903,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
                 }
             }
         }
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-        t0 += n;
     }
-    }
-
-    // a prefetch still in flight (the loop ended early) completes before exit
-    if (prefetched) tc::mbar_wait(s_tbar, tphase);
-
-    // ---- S_out = Diag(f) X
-    if (flags[0] == 0 && p.S_out && T > 0) {
-        const int i = row;
-        for (int cblk = 0; cblk < DVC / 64; ++cblk) {
-            const int col = (DVC / 2) * colhalf + 32 * cblk;
-            float v[32];
-            tc::tmem_ld32(tmem + lane_base + kTmX + col, v);
-            float4 *dst = reinterpret_cast<float4 *>(p.S_out + sbase + (size_t)i * kDV + dv0 + col);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(v[4 * q] * fprev[i], v[4 * q + 1] * fprev[i], v[4 * q + 2] * fprev[i],
-                                     v[4 * q + 3] * fprev[i]);
-        }
-    }
-    if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
-    if (flags[0] != 0 && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
     tc::fence_before_sync();
     __syncthreads();
+    if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
+    if ((flags[0] != 0 || flags[3] != 0) && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
+    // no CTA leaves while its peer may still write into its shared memory
+    tc::cluster_sync();
 }
 
 // ---------------------------------------------------------------------------
@@ -1129,7 +1229,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                     for (int s = 0; s < i; ++s) acc += Lr[i][s] * x[s];
                     if (i > j) x[i] = -acc;
                 }
-                asm volatile("bar.sync 1, 64;" ::: "memory");
+                asm volatile("bar.sync 2, 64;" ::: "memory");
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     if (i >= j) lw[(o + i) * kLW + o + j] = x[i];
@@ -1200,10 +1300,6 @@ size_t fwd_tc_workspace_bytes(int B, int H, int T) {
     return nwin * kWinBytes + ((nwin * sizeof(int) + 1023) & ~(size_t)1023);
 }
 
-size_t fwd_tc_smem_bytes(int dvc) {
-    return (dvc == 128 ? (size_t)Smem<128>::TOTAL : (size_t)Smem<64>::TOTAL) + 1024;
-}
-
 bool fwd_tc_supported(int dtype, int dk, int dv, int chunk) {
     return dtype == GDELTA_BF16 && dk == 128 && dv == 128 && chunk == 64;
 }
@@ -1222,6 +1318,7 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     int *wflags = (int *)(ws + nwin * kWinBytes);
     p.ws = ws;
     p.wflags = wflags;
+
     const size_t ismem = (size_t)IntraSmem::TOTAL + 1024;
     cudaError_t e = cudaFuncSetAttribute(gdn2_chunk_intra_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)ismem);
@@ -1229,10 +1326,11 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     gdn2_chunk_intra_tc_kernel<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem = fwd_tc_smem_bytes(128);
-    e = cudaFuncSetAttribute(gdn2_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = (size_t)ChainSmem::TOTAL + 1024;
+    e = cudaFuncSetAttribute(gdn2_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    gdn2_fwd_tc_kernel<128><<<fp.B * fp.H, kThreads, smem, stream>>>(p);
+    // clusters of two CTAs (value-column halves of one head), set by the kernel's attribute
+    gdn2_fwd_tc_kernel<<<2 * fp.B * fp.H, kChainThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

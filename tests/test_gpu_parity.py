@@ -232,6 +232,22 @@ def test_tc_fast_decay_shortens_chunks(u):
     _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
 
 
+def test_tc_mixed_fast_and_shortened_windows():
+    """Windows whose decay span fits one 64-token chunk interleave with windows
+    that must be shortened (two in a row, a single one, and the ragged tail):
+    the chain switches between precomputed window tiles and its own shorter
+    chunks, and a shortened window borrows the other window buffer as scratch."""
+    shape = synth.GdnShape(B=2, T=64 * 7 + 17, H=2, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=11)
+    inp = synth.generate(shape)
+    la = inp["log_alpha"].clone()
+    for w in (1, 2, 4, 7):
+        la[:, 64 * w: 64 * (w + 1)] *= 40.0
+    inp["log_alpha"] = la
+    y, S, o = gpu_fwd(inp, path="tc")
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, _ref(inp, heads), heads, TOL_BF16)
+
+
 def test_tc_state_in_and_in_place():
     import channel_gated_delta_b200 as gd
     shape = synth.GdnShape(B=2, T=150, H=3, dk=128, dv=128, dtype="bf16", seed=8)
