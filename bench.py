@@ -297,7 +297,10 @@ def run_ours(args, rank, local, world):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "gdn2_fwd_tc_kernel" if path == "tc" else "gdn2_fwd_simt_kernel",
+            # the timed unit is one gdelta_fwd_chunked call: on the tensor-core path
+            # the intra-chunk kernel followed by the chain kernel
+            "kernel": ("gdelta_fwd_chunked = gdn2_chunk_intra_tc_kernel + gdn2_fwd_tc_kernel" if path == "tc"
+                       else "gdn2_fwd_simt_kernel"),
             "achieved": achieved,
             "peak": hbm,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
