@@ -1051,8 +1051,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         }
         const int n = wend - t0;
 
-        // ---- operand tiles: P operands to shared memory; Qp, Kc, K^c and the
-        // pivot vectors straight to the window record
+        // ---- operand tiles: P operands to shared memory (Qp, Kc and K^c reach the
+        // record from there by bulk copy); the pivot vectors straight to the record
         {
             const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
             const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
@@ -1118,9 +1118,6 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 *(uint2 *)(sm + L::AP + off_b) = uqp;
                 *(uint2 *)(sm + L::BP + off_t) = ukc;
                 *(uint2 *)(sm + L::BP + off_b) = ukh;
-                *(uint2 *)(rec + kWinAP + off_b) = uqp;
-                *(uint2 *)(rec + kWinBP + off_t) = ukc;
-                *(uint2 *)(rec + kWinBP + off_b) = ukh;
             }
             // the exact diagonals q~_t.k_t and q~_t.(b*k)_t of Aq / Bq
             const float dsum = reduce_scatter16(dg, lane);
@@ -1142,13 +1139,18 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         tc::fence_proxy_async();
         __syncthreads();
 
-        // ---- P = [Kp; Qp] [Kc; K^c]^T
+        // ---- P = [Kp; Qp] [Kc; K^c]^T; the record's [Kc; K^c] tile and the Qp rows
+        // of [W'; Qp] are copied out of the same shared-memory tiles meanwhile
         if (tid == 0) {
             tc::fence_after_sync();
             const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
             for (int ks = 0; ks < kDK / 16; ++ks)
                 tc::mma_f16(tmem, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id, ks > 0);
             tc::mma_commit(s_mbar);
+            tc::bulk_s2g(rec + kWinBP, s_bp, 128 * 256);
+            tc::bulk_s2g(rec + kWinAP + 64 * 128, s_ap + 64 * 128, 64 * 128);                 // Qp, columns 0-63
+            tc::bulk_s2g(rec + kWinAP + 128 * 128 + 64 * 128, s_ap + 128 * 128 + 64 * 128, 64 * 128);  // columns 64-127
+            tc::bulk_commit();
         }
         // V^ = w*v -> window record (the identity padding past n is zero)
 #pragma unroll
@@ -1168,7 +1170,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         }
         if (!wait_mma()) break;
 
-        // ---- masks; M -> MM (shared), L -> fp32 (over BP), Aq / Bq -> record.
+        // ---- masks; M -> MM (shared), L -> fp32 (over BP), Aq / Bq -> staged over
+        // the Qp rows of AP (in the record's byte layout) and copied to the record.
         // This warp's rows are tokens t in [32 tb2, 32 tb2 + 32): column block hf
         // below the diagonal block is kept whole, above it zeroed, and only the
         // diagonal block is masked element by element.
@@ -1178,7 +1181,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             const int tb2 = warp & 1;
             float v[2][32];
             tc::tmem_ld32x2(tmem + lane_base + 64 * colhalf, tmem + lane_base + 64 * colhalf + 32, v[0], v[1]);
-            // all warps have read P; BP may now be overwritten with L
+            // all warps have read P and the bulk copies have read BP and the Qp rows:
+            // both may now be overwritten
+            if (tid == 0) tc::bulk_wait_read();
             tc::fence_before_sync();
             __syncthreads();
             const float dv_t = upper ? 0.f : (colhalf == 0 ? diagq[t] : diagb[t]);
@@ -1203,12 +1208,18 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 } else if (upper) {
                     store_row32(sm + L::MM, 64, t, 32 * hf, v[hf]);
                 } else {
-                    store_row32(rec + kWinANAB, 192, colhalf == 0 ? 64 + t : 128 + t, 32 * hf, v[hf]);
+                    store_row32(sm + L::AP + (colhalf == 0 ? 64 * 128 : 128 * 128 + 64 * 128), 64, t, 32 * hf, v[hf]);
                 }
             }
         }
+        tc::fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+            tc::bulk_s2g(rec + kWinANAB + 64 * 128, s_ap + 64 * 128, 64 * 128);                 // Aq
+            tc::bulk_s2g(rec + kWinANAB + 128 * 128, s_ap + 128 * 128 + 64 * 128, 64 * 128);    // Bq
+            tc::bulk_commit();
+        }
 
         // ---- T^-1 = (I + L)^-1 (divide and conquer, fp32)
         {
@@ -1264,7 +1275,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         }
         if (!wait_mma()) break;
 
-        // ---- W' -> record rows 0-63 of [W'; Qp]; N -> record rows 0-63 of [N; Aq; Bq]
+        // ---- W' -> staged over Kp (rows 0-63 of AP), N -> over M; both copied to
+        // rows 0-63 of the record's [W'; Qp] and [N; Aq; Bq]
         {
             const int t = 16 * (warp & 3) + lane;
             const bool valid = lane < 16;
@@ -1275,18 +1287,28 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     range_max = fmaxf(range_max, maxabs(v[hf], 32));
-                    store_row32(rec + kWinAP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
+                    store_row32(sm + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
                 }
             }
             float nv[32];
             tc::tmem_ld32(tmem + lane_base + kItmN + 32 * colhalf, nv);
             if (valid) {
                 range_max = fmaxf(range_max, maxabs(nv, 32));
-                store_row32(rec + kWinANAB, 192, t, 32 * colhalf, nv);
+                store_row32(sm + L::MM, 64, t, 32 * colhalf, nv);
             }
         }
-        if (tid == 0) wflags[wi] = 0;
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            tc::bulk_s2g(rec + kWinAP, s_ap, 64 * 128);                              // W', columns 0-63
+            tc::bulk_s2g(rec + kWinAP + 128 * 128, s_ap + 128 * 128, 64 * 128);      // columns 64-127
+            tc::bulk_s2g(rec + kWinANAB, s_mm, 64 * 128);                            // N
+            tc::bulk_commit();
+            wflags[wi] = 0;
+        }
     } while (false);
+    // the record's bulk copies complete before the CTA's shared memory goes away
+    if (tid == 0) tc::bulk_wait_all();
 
     if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
     if (flags[0] != 0 && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
