@@ -22,6 +22,7 @@ one JSON line with the max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -53,6 +54,10 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # profiling aid: a smaller case of the same workload (fewer batch rows) for
+    # ncu captures that must stay small; the bench line itself uses the default
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch rows (for profiler captures only)")
     return ap.parse_args()
 
 
@@ -197,6 +202,8 @@ def run_ours(args, rank, local, world):
 
     dev = torch.device("cuda", local)
     shape = synth.CONFIGS[WORKLOAD]
+    if args.batch > 0:
+        shape = dataclasses.replace(shape, B=args.batch)
     B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
     host = synth.generate(shape, seed=shape.seed + 1000 * rank)
     d = {k: v.to(dev) for k, v in host.items()}
