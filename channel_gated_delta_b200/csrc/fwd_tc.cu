@@ -258,8 +258,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     int *pflag = (int *)(sm + L::PART + 512);     // [2] the peer's abort flags
     volatile int *flags = (volatile int *)(sm + L::MISC + 96);  // [0] local abort, [1] chosen n, [2] log2 of the chunk, [3] agreed abort
     int *info = (int *)(sm + L::MISC + 112);      // per O slot: t0, n, done
+    volatile int *req = (volatile int *)(sm + L::MISC + 176);  // record requests: [2] x (window, buffer)
     const uint32_t s_mbar = tc::smem_u32(mbar), s_rbar = s_mbar + 8, s_xbar = s_mbar + 24;
     const uint32_t s_ibar = s_mbar + 40, s_obar = s_mbar + 56, s_fbar = s_mbar + 72;
+    const uint32_t s_lq = s_mbar + 144, s_lfree = s_mbar + 160;  // record request posted / slot read
     const uint32_t peer_rank = crank ^ 1u;
     const uint32_t r_peer = tc::mapa(tc::smem_u32(peer), peer_rank);
     const uint32_t r_pflag = tc::mapa(tc::smem_u32(pflag), peer_rank);
@@ -273,6 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     }
     if (tid == 0) {
         for (int i = 0; i < 11; ++i) tc::mbar_init(s_mbar + 8 * i, 1);
+        for (int i = 0; i < 4; ++i) tc::mbar_init(s_lq + 8 * i, 1);
         tc::mbar_arrive_expect_tx(s_xbar, 65 * 4);   // the peer's sums of chunk 0 (64 rows and a flag)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
@@ -293,6 +296,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     const int colhalf = warp >> 2;                                  // 32-column half of this CTA's 64
     float range_max = 0.f;
 
+    const int NW = p.NW;
+    const size_t wbase = (size_t)head * NW;
+    // Record copies are issued by one lane of warp 8, which executes no proxy
+    // fence: a thread that has bulk copies in flight and then fences the async
+    // proxy (as the state warps do after staging operand tiles) waits for those
+    // copies, which would tie every window to the record two windows ahead.
+    auto issue_rec = [&](int w, int b) {         // window w's record -> buffer b
+        const uint8_t *rec = p.ws + (wbase + w) * kWinBytes;
+        uint8_t *dst = sm + b * L::BUF;
+        const uint32_t bar = s_rbar + 8u * b;
+        tc::mbar_arrive_expect_tx(bar, L::BUF);
+        tc::bulk_g2s(tc::smem_u32(dst + L::AP), rec + kWinAP, 128 * 256, bar);
+        tc::bulk_g2s(tc::smem_u32(dst + L::BP), rec + kWinBP, 128 * 256, bar);
+        tc::bulk_g2s(tc::smem_u32(dst + L::ANAB), rec + kWinANAB, 192 * 128, bar);
+        tc::bulk_g2s(tc::smem_u32(dst + L::VH), rec + kWinVH + crank * (64 * 128), 64 * 128, bar);
+        tc::bulk_g2s(tc::smem_u32(dst + L::EV), rec + kWinVEC, 2 * 128 * 4, bar);
+    };
+    static_assert(L::BUF == 2 * 128 * 256 + 192 * 128 + 64 * 128 + 1024, "record buffer = bytes of one record copy");
+
     if (warp < 8) {
         // Wait for the MMAs committed so far; a timeout marks a local abort.
         auto wait_mma = [&]() -> bool {
@@ -303,28 +325,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             return flags[0] == 0;
         };
 
-        const int NW = p.NW;
-        const size_t wbase = (size_t)head * NW;
         auto win_fast = [&](int w) -> bool { return p.ws != nullptr && w < NW && p.wflags[wbase + w] == 0; };
-        auto issue_rec = [&](int w, int b) {         // thread 0: window w's record -> buffer b
-            const uint8_t *rec = p.ws + (wbase + w) * kWinBytes;
-            uint8_t *dst = sm + b * L::BUF;
-            const uint32_t bar = s_rbar + 8u * b;
-            tc::fence_proxy_async();
-            tc::mbar_arrive_expect_tx(bar, L::BUF);
-            tc::bulk_g2s(tc::smem_u32(dst + L::AP), rec + kWinAP, 128 * 256, bar);
-            tc::bulk_g2s(tc::smem_u32(dst + L::BP), rec + kWinBP, 128 * 256, bar);
-            tc::bulk_g2s(tc::smem_u32(dst + L::ANAB), rec + kWinANAB, 192 * 128, bar);
-            tc::bulk_g2s(tc::smem_u32(dst + L::VH), rec + kWinVH + crank * (64 * 128), 64 * 128, bar);
-            tc::bulk_g2s(tc::smem_u32(dst + L::EV), rec + kWinVEC, 2 * 128 * 4, bar);
+        // thread 0: post a record request (window w into buffer b; w < 0 stops the loader)
+        uint32_t nreq = 0;
+        auto enqueue = [&](int w, int b) {
+            const uint32_t k = nreq++, sl = k & 1u;
+            if (k >= 2 && !tc::mbar_wait(s_lfree + 8u * sl, ((k >> 1) - 1) & 1u)) flags[0] = 1;
+            req[2 * sl] = w;
+            req[2 * sl + 1] = b;
+            tc::mbar_arrive_local(s_lq + 8u * sl);
         };
-        static_assert(L::BUF == 2 * 128 * 256 + 192 * 128 + 64 * 128 + 1024, "record buffer = bytes of one record copy");
 
         int loaded[2] = {-1, -1};                     // window whose record buffer b holds or receives
         bool inflight[2] = {false, false};            // a copy into buffer b not yet waited for
         for (int b = 0; b < 2; ++b)
             if (win_fast(b)) {
-                if (tid == 0) issue_rec(b, b);
+                if (tid == 0) enqueue(b, b);
                 loaded[b] = b;
                 inflight[b] = true;
             }
@@ -785,7 +801,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         main_sync();
                         if (t0 + n == wend) {
                             if (wflag2 == 0) {
-                                if (tid == 0) issue_rec(w + 2, B);
+                                if (tid == 0) enqueue(w + 2, B);
                                 loaded[B] = w + 2;
                                 inflight[B] = true;
                             } else {
@@ -805,7 +821,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             // (its scratch buffer) is copied again, and this buffer takes window w + 2
             if (!fast && flags[0] == 0) {
                 if (loaded[B ^ 1] == w + 1) {
-                    if (tid == 0) issue_rec(w + 1, B ^ 1);
+                    if (tid == 0) enqueue(w + 1, B ^ 1);
                     inflight[B ^ 1] = true;
                 }
             }
@@ -818,6 +834,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             info[4 * slot + 2] = 1;
             tc::mbar_arrive_local(s_ibar + 8u * slot);
         }
+        if (tid == 0) enqueue(-1, 0);
         // copies still in flight (the loop ended early) complete before exit
         for (int b = 0; b < 2; ++b)
             if (inflight[b]) tc::mbar_wait(s_rbar + 8u * b, rphase[b]);
@@ -833,6 +850,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             for (int q = 0; q < 8; ++q)
                 dst[q] = make_float4(v[4 * q] * fprev[i], v[4 * q + 1] * fprev[i], v[4 * q + 2] * fprev[i],
                                      v[4 * q + 3] * fprev[i]);
+        }
+    } else if (warp == 8) {
+        // ---- record loader: one lane serves the state warps' requests in order
+        if (lane == 0) {
+            for (uint32_t k = 0;; ++k) {
+                const uint32_t sl = k & 1u;
+                bool got = false;
+                for (int tries = 0; tries < 64 && !got; ++tries) {
+                    got = tc::mbar_wait(s_lq + 8u * sl, (k >> 1) & 1u);
+                    if (!got && (flags[0] != 0 || flags[3] != 0)) break;
+                }
+                if (!got) break;
+                const int w = req[2 * sl], b = req[2 * sl + 1];
+                tc::mbar_arrive_local(s_lfree + 8u * sl);
+                if (w < 0) break;
+                issue_rec(w, b);
+            }
         }
     } else if (warp >= 10) {
         // ---- readout warps: O (TMEM lanes 64-127) -> RMS norm over d_v (both
