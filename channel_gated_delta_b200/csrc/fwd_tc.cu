@@ -886,10 +886,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             // the gate of this row, fetched while the chunk's products run
             const bool live = et < n;
             const size_t gi = (((size_t)bb * T + t0 + et) * H + h) * kDV + dv0;
+            // 32-byte accesses when the tensors allow them: the row pieces of a chunk
+            // are 4 KB apart, and full-sector accesses keep the SM's memory queue
+            // short for the record copies that share it
+            const bool a32 = ((reinterpret_cast<uintptr_t>(p.g) | reinterpret_cast<uintptr_t>(p.y) |
+                               reinterpret_cast<uintptr_t>(p.o_raw)) & 31u) == 0;
             uint4 gq[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                gq[q] = live ? __ldg(reinterpret_cast<const uint4 *>(p.g + gi) + q) : make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 8; ++q) gq[q] = make_uint4(0, 0, 0, 0);
+            if (live) {
+                if (a32) {
+#pragma unroll
+                    for (int q = 0; q < 8; q += 2) tc::ld_global_nc_v8(p.g + gi + 8 * q, gq[q], gq[q + 1]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) gq[q] = __ldg(reinterpret_cast<const uint4 *>(p.g + gi) + q);
+                }
+            }
             bool ok = true;
             if (et == 0) ok = tc::mbar_wait(s_obar + 8u * slot, ph);
             asm volatile("bar.sync 3, 64;" ::: "memory");
@@ -899,7 +912,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             tc::tmem_ld32x2(tmem + lane_base + ro, tmem + lane_base + ro + 32, ov[0], ov[1]);
             tc::fence_before_sync();
             asm volatile("bar.sync 3, 64;" ::: "memory");
-            if (et == 0) tc::mbar_arrive_local(s_fbar + 8u * slot);   // the slot may take a new chunk
+            // the slot may take a new chunk; a releasing arrival would first wait for
+            // this thread's y stores of the previous chunk to reach L2
+            if (et == 0) tc::mbar_arrive_local_relaxed(s_fbar + 8u * slot);
             float ss = 0.f;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
@@ -917,22 +932,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             if (flags[3] != 0) break;
             if (live) {
                 const float inv = rsqrtf((ss + peer[slot * 64 + et]) / kDV + p.eps);
+                uint4 yq[8];
 #pragma unroll
                 for (int q8 = 0; q8 < 8; ++q8) {
-                    float gg[8], yy[8];
+                    float gg[8];
                     bf16x8_to_f(gq[q8], gg);
                     const float *o8 = &ov[q8 >> 2][8 * (q8 & 3)];
+                    __nv_bfloat162 *hb = reinterpret_cast<__nv_bfloat162 *>(&yq[q8]);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) yy[e] = gg[e] * o8[e] * inv;
-                    uint4 u;
-                    __nv_bfloat162 *hb = reinterpret_cast<__nv_bfloat162 *>(&u);
+                    for (int e = 0; e < 4; ++e)
+                        hb[e] = __floats2bfloat162_rn(gg[2 * e] * o8[2 * e] * inv, gg[2 * e + 1] * o8[2 * e + 1] * inv);
+                }
+                if (a32) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) hb[e] = __floats2bfloat162_rn(yy[2 * e], yy[2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(p.y + gi + 8 * q8) = u;
-                    if (p.o_raw) {
-                        float4 *dst = reinterpret_cast<float4 *>(p.o_raw + gi + 8 * q8);
-                        dst[0] = make_float4(o8[0], o8[1], o8[2], o8[3]);
-                        dst[1] = make_float4(o8[4], o8[5], o8[6], o8[7]);
+                    for (int q8 = 0; q8 < 8; q8 += 2) tc::st_global_v8(p.y + gi + 8 * q8, yq[q8], yq[q8 + 1]);
+                } else {
+#pragma unroll
+                    for (int q8 = 0; q8 < 8; ++q8) *reinterpret_cast<uint4 *>(p.y + gi + 8 * q8) = yq[q8];
+                }
+                if (p.o_raw) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        const float *o8 = &ov[q8 >> 2][8 * (q8 & 3)];
+                        const uint4 lo = make_uint4(__float_as_uint(o8[0]), __float_as_uint(o8[1]), __float_as_uint(o8[2]),
+                                                    __float_as_uint(o8[3]));
+                        const uint4 hi = make_uint4(__float_as_uint(o8[4]), __float_as_uint(o8[5]), __float_as_uint(o8[6]),
+                                                    __float_as_uint(o8[7]));
+                        if (a32) {
+                            tc::st_global_v8(p.o_raw + gi + 8 * q8, lo, hi);
+                        } else {
+                            reinterpret_cast<uint4 *>(p.o_raw + gi + 8 * q8)[0] = lo;
+                            reinterpret_cast<uint4 *>(p.o_raw + gi + 8 * q8)[1] = hi;
+                        }
                     }
                 }
             }

@@ -208,6 +208,13 @@ __device__ __forceinline__ void mbar_arrive_local(uint32_t mbar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 
+// One arrival on a local mbarrier without release semantics: it does not wait
+// for this thread's earlier global stores to be performed.  For handing back
+// a TMEM region whose reads completed (tcgen05.wait::ld) before the arrival.
+__device__ __forceinline__ void mbar_arrive_local_relaxed(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
 // One expected arrival that also announces `bytes` of asynchronous transfers.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
@@ -299,6 +306,19 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t mbar, uint32_t parity
 // All threads of all CTAs of the cluster.
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 32-byte global accesses (sm_100): one full sector per thread and instruction;
+// the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *p, const uint4 &a, const uint4 &b) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+__device__ __forceinline__ void ld_global_nc_v8(const void *p, uint4 &a, uint4 &b) {
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
