@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-forms", action="store_true",
+                    help="skip the forward timings of the reduced gate forms")
     # profiling aid: a smaller case of the same workload (fewer batch rows) for
     # ncu captures that must stay small; the bench line itself uses the default
     ap.add_argument("--batch", type=int, default=0,
@@ -159,10 +161,16 @@ class ClockSampler:
                 "samples": len(rows), "reasons": reasons}
 
 
-def fwd_bytes(B, T, H, dk, dv, tok_bytes):
+def fwd_bytes(B, T, H, dk, dv, tok_bytes, z=True, beta=False, decay_tok=False):
     """Algorithmic HBM bytes of one chunked-forward launch: q,k,z,b (d_k) and
-    v,w,g (d_v) tokens, fp32 log-decay, y, the fp32 state read and written."""
-    per_token_head = 4 * dk * tok_bytes + 3 * dv * tok_bytes + 4 * dk + dv * tok_bytes
+    v,w,g (d_v) tokens, fp32 log-decay, y, the fp32 state read and written.
+    Reduced gate forms: no z; one beta per token and head in place of the b
+    and w rows; one fp32 log-decay per token and head."""
+    n_dk = 2 + (1 if z else 0) + (0 if beta else 1)          # q, k [, z] [, b]
+    n_dv = 2 + (0 if beta else 1)                            # v, g [, w]
+    per_token_head = (n_dk * dk + n_dv * dv + dv) * tok_bytes + (4 if decay_tok else 4 * dk)
+    if beta:
+        per_token_head += tok_bytes
     return B * T * H * per_token_head + 2 * B * H * dk * dv * 4 + H * dk * 4
 
 
@@ -272,6 +280,9 @@ def run_ours(args, rank, local, world):
     # ---- decode-only measurement (batch 64 x 16 heads, L2 flushed between steps)
     dec = run_decode(args, dev, stream, rank, world) if args.decode_steps > 0 else None
 
+    # ---- forward alone on the reduced gate forms (same workload shape)
+    forms = None if args.no_forms else run_forms(args, gd, d, shape, dev, stream, ws, world)
+
     # ---- end to end through the public API with host buffers
     e2e = None if args.no_e2e else run_e2e(args, gd, host, dev, stream, shape, world, path)
 
@@ -324,6 +335,7 @@ def run_ours(args, rank, local, world):
         "gpu_launches": (4 if path == "tc" else 3) * args.steps,
         "clocks": clk,
         "decode": dec,
+        "forms": forms,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -381,6 +393,59 @@ def run_decode(args, dev, stream, rank, world):
         "l2": "256 MB buffer written between timed steps (state evicted)",
         "state_init": "random N(0, 0.05^2) state (timing does not depend on values)",
     }
+
+
+FORMS = {
+    # Muir readout with the static profile only (no dynamic z)
+    "static_gain": dict(z=False, beta=False, decay_tok=False),
+    # KDA: one beta for erase and write, per-channel decay
+    "kda": dict(z=True, beta=True, decay_tok=False),
+    # Gated DeltaNet: one beta and one scalar decay per token, no z
+    "gdn": dict(z=False, beta=True, decay_tok=True),
+}
+
+
+def run_forms(args, gd, d, shape, dev, stream, ws, world):
+    """Times gdelta_fwd_chunked alone on each reduced gate form, inputs made
+    from the workload's tensors (beta = channel 0 of w, the scalar log-decay =
+    channel 0 of log_alpha).  Inputs stay larger than L2 for every form."""
+    B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+    S = torch.empty(B, H, dk, dv, device=dev)
+    y = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    hbm, _ = peaks()
+    out = {}
+    for name, f in FORMS.items():
+        z = d["z"] if f["z"] else None
+        beta = d["w"][..., 0].contiguous() if f["beta"] else None
+        b, w = (None, None) if f["beta"] else (d["b"], d["w"])
+        la = d["log_alpha"][..., 0].contiguous() if f["decay_tok"] else d["log_alpha"]
+
+        def call():
+            gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], b, w, z, d["g"], la, gamma_stat=d["gamma_stat"],
+                                  S_in=S, S_out=S, y=y, chunk=C, path=args.path, workspace=ws,
+                                  stream=stream, beta=beta, decay_per_token=f["decay_tok"])
+
+        for _ in range(3):
+            gd.gdelta_state_init(S, stream=stream)
+            call()
+        torch.cuda.synchronize(dev)
+        if gd.gdelta_get_last_device_error(stream) != 0:
+            raise RuntimeError(f"device status word set during the {name} warm-up")
+        n = max(3, args.steps)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        barrier(world)
+        for i in range(n):
+            gd.gdelta_state_init(S, stream=stream)
+            evs[i][0].record(stream)
+            call()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
+        nb = fwd_bytes(B, T, H, dk, dv, 2, **f)
+        gbs = nb / (ms * 1e-3) / 1e9
+        out[name] = {"fwd_ms_median": ms, "tokens_per_s": B * T * world / (ms * 1e-3),
+                     "algorithmic_bytes": nb, "achieved_gbs": gbs, "frac": gbs / hbm, "timed_calls": n}
+    return out
 
 
 def run_e2e(args, gd, host, dev, stream, shape, world, path):

@@ -93,7 +93,7 @@ def gdelta_status_string(status: int) -> str:
 
 
 def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
-                path, workspace) -> _native.FwdArgs:
+                path, workspace, beta=None, decay_per_token=False) -> _native.FwdArgs:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -105,12 +105,14 @@ def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_ra
     ks, vs = (B, T, H, dk), (B, T, H, dv)
     a.q = _dev_ptr(q, "q", dt, ks)
     a.k = _dev_ptr(k, "k", dt, ks)
-    a.z = _dev_ptr(z, "z", dt, ks)
-    a.b = _dev_ptr(b, "b", dt, ks)
+    a.z = _dev_ptr(z, "z", dt, ks, required=False)
+    a.b = _dev_ptr(b, "b", dt, ks, required=beta is None)
     a.v = _dev_ptr(v, "v", dt, vs)
-    a.w = _dev_ptr(w, "w", dt, vs)
+    a.w = _dev_ptr(w, "w", dt, vs, required=beta is None)
     a.g = _dev_ptr(g, "g", dt, vs)
-    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, ks)
+    a.beta = _dev_ptr(beta, "beta", dt, (B, T, H), required=False)
+    a.decay_per_token = int(bool(decay_per_token))
+    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, (B, T, H) if decay_per_token else ks)
     a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
     a.S_in = _dev_ptr(S_in, "S_in", torch.float32, (B, H, dk, dv), required=False)
     a.S_out = _dev_ptr(S_out, "S_out", torch.float32, (B, H, dk, dv), required=False)
@@ -124,16 +126,16 @@ def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_ra
 
 
 def gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
-                               path: str = "auto") -> int:
+                               path: str = "auto", beta=None, decay_per_token: bool = False) -> int:
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
-                    path, None)
+                    path, None, beta, decay_per_token)
     return int(_lib().gdelta_fwd_workspace_bytes(ctypes.byref(a)))
 
 
 def gdelta_fwd_selected_path(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
-                             path: str = "auto") -> str:
+                             path: str = "auto", beta=None, decay_per_token: bool = False) -> str:
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
-                    path, None)
+                    path, None, beta, decay_per_token)
     code = int(_lib().gdelta_fwd_selected_path(ctypes.byref(a)))
     if code < 0:
         raise GdeltaError(2, "gdelta_fwd_selected_path")
@@ -153,9 +155,15 @@ def gdelta_state_init(S: torch.Tensor, S_src: Optional[torch.Tensor] = None, str
 
 def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=None, S_out=None,
                        y=None, o_raw=None, chunk: int = 64, eps: float = 1e-6, path: str = "auto",
-                       workspace=None, return_state: bool = True, stream=None
+                       workspace=None, return_state: bool = True, stream=None, beta=None,
+                       decay_per_token: bool = False
                        ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked forward over [B,T,H,d] tokens.  Returns (y, S_out).
+
+    Reduced gate forms: ``z`` may be None (no dynamic readout gain);
+    ``beta`` [B,T,H] replaces ``b`` and ``w`` (pass them as None) with one
+    gate per token and head; ``decay_per_token`` takes ``log_alpha`` as
+    [B,T,H].  Together these give the KDA and Gated DeltaNet special cases.
 
     Outputs not passed in are allocated with torch on q's device; S_out is
     only allocated when ``return_state``.  ``workspace`` (uint8 CUDA tensor) is
@@ -168,18 +176,24 @@ def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=
     if S_out is None and return_state:
         S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     if workspace is None:
-        need = gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, chunk=chunk, path=path)
+        need = gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, chunk=chunk, path=path,
+                                          beta=beta, decay_per_token=decay_per_token)
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
-                    path, workspace)
+                    path, workspace, beta, decay_per_token)
     _check(_lib().gdelta_fwd_chunked(ctypes.byref(a), _stream(stream)), "gdelta_fwd_chunked")
     return y, S_out
 
 
 def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=None, o_raw=None,
-                       eps: float = 1e-6, stream=None) -> torch.Tensor:
-    """One token per (batch, head): S [B,H,dk,dv] fp32 updated in place; returns y [B,H,dv]."""
+                       eps: float = 1e-6, stream=None, beta=None,
+                       decay_per_token: bool = False) -> torch.Tensor:
+    """One token per (batch, head): S [B,H,dk,dv] fp32 updated in place; returns y [B,H,dv].
+
+    ``z``, ``beta`` and ``decay_per_token`` as in gdelta_fwd_chunked, with
+    beta [B,H] and a per-token log_alpha [B,H].
+    """
     B, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -192,12 +206,14 @@ def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=
     ks, vs = (B, H, dk), (B, H, dv)
     a.q = _dev_ptr(q, "q", dt, ks)
     a.k = _dev_ptr(k, "k", dt, ks)
-    a.z = _dev_ptr(z, "z", dt, ks)
-    a.b = _dev_ptr(b, "b", dt, ks)
+    a.z = _dev_ptr(z, "z", dt, ks, required=False)
+    a.b = _dev_ptr(b, "b", dt, ks, required=beta is None)
     a.v = _dev_ptr(v, "v", dt, vs)
-    a.w = _dev_ptr(w, "w", dt, vs)
+    a.w = _dev_ptr(w, "w", dt, vs, required=beta is None)
     a.g = _dev_ptr(g, "g", dt, vs)
-    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, ks)
+    a.beta = _dev_ptr(beta, "beta", dt, (B, H), required=False)
+    a.decay_per_token = int(bool(decay_per_token))
+    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, (B, H) if decay_per_token else ks)
     a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
     a.S = _dev_ptr(S, "S", torch.float32, (B, H, dk, dv))
     a.y = _dev_ptr(y, "y", dt, vs)

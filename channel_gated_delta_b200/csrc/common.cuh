@@ -31,6 +31,9 @@ __device__ __forceinline__ float warp_sum(float x) {
 // Device status codes written by kernels that detect a run-time fault.
 enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2 };
 
+// Gate and decay forms (gdelta.h): z may be null (read as 0); beta, when
+// non-null, replaces b and w (one value per token and head); decay_tok = 1
+// means log_alpha holds one value per token and head.
 struct FwdParams {
     int B, T, H, dk, dv, C;
     const void *q, *k, *z, *b, *v, *w, *g;
@@ -39,6 +42,8 @@ struct FwdParams {
     void *y;
     float *o_raw;
     float eps;
+    const void *beta;
+    int decay_tok;
     int *status;
 };
 
@@ -50,6 +55,8 @@ struct DecodeParams {
     void *y;
     float *o_raw;
     float eps;
+    const void *beta;
+    int decay_tok;
 };
 
 // Launchers (return cudaError_t of the launch).

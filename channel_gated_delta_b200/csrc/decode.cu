@@ -62,14 +62,14 @@ __global__ void __launch_bounds__(256, 4) gdn2_decode_kernel(DecodeParams p) {
     }
 
     const T *q = (const T *)p.q, *k = (const T *)p.k, *z = (const T *)p.z, *b = (const T *)p.b;
-    const T *v = (const T *)p.v, *w = (const T *)p.w;
+    const T *v = (const T *)p.v, *w = (const T *)p.w, *beta = (const T *)p.beta;
     float cb = 0.f, ck = 0.f;
     for (int i = tid; i < DK; i += NT) {
         const float ki = ldf(k, kbase + i);
-        const float bi = ldf(b, kbase + i);
-        const float al = expf(p.la[kbase + i]);
+        const float bi = beta ? ldf(beta, head) : ldf(b, kbase + i);
+        const float al = expf(p.decay_tok ? p.la[head] : p.la[kbase + i]);
         const float gs = p.gs ? p.gs[(size_t)h * DK + i] : 1.f;
-        const float qt = ldf(q, kbase + i) * gs * two_sigmoid(ldf(z, kbase + i));
+        const float qt = ldf(q, kbase + i) * gs * two_sigmoid(z ? ldf(z, kbase + i) : 0.f);
         s_k[i] = ki;
         s_kh[i] = bi * ki;
         s_alpha[i] = al;
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256, 4) gdn2_decode_kernel(DecodeParams p) {
         cb += qt * bi * ki;
         ck += qt * ki;
     }
-    for (int j = tid; j < DV; j += NT) s_vh[j] = ldf(w, vbase + j) * ldf(v, vbase + j);
+    for (int j = tid; j < DV; j += NT) s_vh[j] = (beta ? ldf(beta, head) : ldf(w, vbase + j)) * ldf(v, vbase + j);
     cb = warp_sum(cb);
     ck = warp_sum(ck);
     if ((tid & 31) == 0) {

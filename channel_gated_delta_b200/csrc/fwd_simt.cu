@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256) gdn2_fwd_simt_kernel(FwdParams p) {
     const int head = blockIdx.x;
     const int bb = head / H, h = head % H;
     const T *q = (const T *)p.q, *k = (const T *)p.k, *z = (const T *)p.z, *b = (const T *)p.b;
-    const T *v = (const T *)p.v, *w = (const T *)p.w, *g = (const T *)p.g;
+    const T *v = (const T *)p.v, *w = (const T *)p.w, *g = (const T *)p.g, *beta = (const T *)p.beta;
 
     // S_0
     const size_t sbase = (size_t)head * dk * dv;
@@ -93,12 +93,13 @@ __global__ void __launch_bounds__(256) gdn2_fwd_simt_kernel(FwdParams p) {
             const int t = e / dk, i = e % dk;
             float kv = 0.f, bv = 0.f, qv = 0.f, lv = 0.f;
             if (t < n) {
-                const size_t gi = (((size_t)bb * T_ + t0 + t) * H + h) * dk + i;
+                const size_t gt = ((size_t)bb * T_ + t0 + t) * H + h;   // token and head
+                const size_t gi = gt * dk + i;
                 kv = ldf(k, gi);
-                bv = ldf(b, gi);
+                bv = beta ? ldf(beta, gt) : ldf(b, gi);
                 const float gs = p.gs ? p.gs[(size_t)h * dk + i] : 1.f;
-                qv = ldf(q, gi) * gs * two_sigmoid(ldf(z, gi));
-                lv = p.la[gi];
+                qv = ldf(q, gi) * gs * two_sigmoid(z ? ldf(z, gi) : 0.f);
+                lv = p.decay_tok ? p.la[gt] : p.la[gi];
             }
             sk[t * dkp + i] = kv;
             skh[t * dkp + i] = bv * kv;
@@ -109,8 +110,9 @@ __global__ void __launch_bounds__(256) gdn2_fwd_simt_kernel(FwdParams p) {
             const int t = e / dv, j = e % dv;
             float x = 0.f;
             if (t < n) {
-                const size_t gi = (((size_t)bb * T_ + t0 + t) * H + h) * dv + j;
-                x = ldf(w, gi) * ldf(v, gi);
+                const size_t gt = ((size_t)bb * T_ + t0 + t) * H + h;
+                const size_t gi = gt * dv + j;
+                x = (beta ? ldf(beta, gt) : ldf(w, gi)) * ldf(v, gi);
             }
             svh[t * dv + j] = x;
         }

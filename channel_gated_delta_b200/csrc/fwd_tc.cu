@@ -152,6 +152,8 @@ struct TcParams {
     int *status;
     const uint8_t *ws;       // per-window chunk tiles from the intra kernel, or null
     const int *wflags;       // per-window flag: 0 = tiles valid, 1 = process here
+    const __nv_bfloat16 *beta;   // one gate per token and head standing for both b and w, or null
+    int decay_tok;               // 1: la holds one log-decay per token and head
     int NW;                  // windows of 64 tokens per head
 };
 
@@ -163,6 +165,12 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4 &u, float *f) {
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
+}
+
+// A gate given once per token and head, repeated over four channels as a bf16 quad.
+__device__ __forceinline__ uint2 bf16x4_bcast(const __nv_bfloat16 *p, size_t i) {
+    const uint32_t x = __ldg(reinterpret_cast<const unsigned short *>(p) + i);
+    return make_uint2(x | (x << 16), x | (x << 16));
 }
 
 __device__ __forceinline__ uint4 pack8(const float *f) {
@@ -394,14 +402,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     for (int u = 0; u < 8; ++u) {
                         const int t = tb + u;
                         const bool in = t0 + t < wend;
-                        const size_t gk = (((size_t)bb * T + t0 + t) * H + h) * kDK + c4;
+                        const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gk = gt * kDK + c4;
                         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (in) x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                        if (in) {
+                            if (p.decay_tok) {
+                                const float s = __ldg(p.la + gt);
+                                x = make_float4(s, s, s, s);
+                            } else {
+                                x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                            }
+                        }
                         la[u][0] = x.x; la[u][1] = x.y; la[u][2] = x.z; la[u][3] = x.w;
                         kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
                         kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-                        kq[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-                        kq[u][3] = in ? __ldg(reinterpret_cast<const uint2 *>(p.b + gk)) : make_uint2(0, 0);
+                        kq[u][2] = in && p.z ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+                        kq[u][3] = !in ? make_uint2(0, 0)
+                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
                     }
                     // inclusive scan over tokens: within this warp's 8 tokens, then across warps
 #pragma unroll
@@ -468,9 +484,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     for (int u = 0; u < 8; ++u) {
                         const int t = tb + u;
                         const bool in = t0 + t < wend && vlane;
-                        const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + dv0 + c4;
+                        const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gv = gt * kDV + dv0 + c4;
                         vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                        vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
+                        vw[u][1] = !in ? make_uint2(0, 0)
+                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
                     }
                     main_sync();
                     n = flags[1];
@@ -1003,6 +1020,9 @@ constexpr uint32_t kItmW = 0;      // W' (M=64) reuses the columns of P after it
 constexpr uint32_t kItmN = 128;    // N  (M=64)
 }  // namespace
 
+// kGates: the gate inputs may come in their reduced forms (one beta for b and w,
+// one log-decay per token, no z); false compiles the plain per-channel loads.
+template <bool kGates>
 __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
     using L = IntraSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1066,14 +1086,22 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         for (int u = 0; u < 8; ++u) {
             const int t = tb + u;
             const bool in = t0 + t < wend;
-            const size_t gk = (((size_t)bb * T + t0 + t) * H + h) * kDK + c4;
+            const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gk = gt * kDK + c4;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (in) x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+            if (in) {
+                if (kGates && p.decay_tok) {
+                    const float s = __ldg(p.la + gt);
+                    x = make_float4(s, s, s, s);
+                } else {
+                    x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                }
+            }
             la[u][0] = x.x * kLog2e; la[u][1] = x.y * kLog2e; la[u][2] = x.z * kLog2e; la[u][3] = x.w * kLog2e;
             kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
             kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-            kq[u][2] = in ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-            kq[u][3] = in ? __ldg(reinterpret_cast<const uint2 *>(p.b + gk)) : make_uint2(0, 0);
+            kq[u][2] = in && (!kGates || p.z) ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+            kq[u][3] = !in ? make_uint2(0, 0)
+                      : kGates && p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
         }
 #pragma unroll
         for (int u = 1; u < 8; ++u)
@@ -1197,9 +1225,10 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         for (int u = 0; u < 8; ++u) {
             const int t = tb + u;
             const bool in = t0 + t < wend;
-            const size_t gv = (((size_t)bb * T + t0 + t) * H + h) * kDV + c4;
+            const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gv = gt * kDV + c4;
             vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-            vw[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.w + gv)) : make_uint2(0, 0);
+            vw[u][1] = !in ? make_uint2(0, 0)
+                      : kGates && p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
         }
         tc::fence_proxy_async();
         __syncthreads();
@@ -1398,6 +1427,7 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.b = (const __nv_bfloat16 *)fp.b; p.v = (const __nv_bfloat16 *)fp.v; p.w = (const __nv_bfloat16 *)fp.w;
     p.g = (const __nv_bfloat16 *)fp.g;
     p.la = fp.la; p.gs = fp.gs; p.S_in = fp.S_in; p.S_out = fp.S_out;
+    p.beta = (const __nv_bfloat16 *)fp.beta; p.decay_tok = fp.decay_tok;
     p.y = (__nv_bfloat16 *)fp.y; p.o_raw = fp.o_raw; p.eps = fp.eps; p.status = fp.status;
     p.NW = (fp.T + kC - 1) / kC;
     const size_t nwin = (size_t)fp.B * fp.H * p.NW;
@@ -1407,10 +1437,11 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.wflags = wflags;
 
     const size_t ismem = (size_t)IntraSmem::TOTAL + 1024;
-    cudaError_t e = cudaFuncSetAttribute(gdn2_chunk_intra_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ismem);
+    const bool gates = p.beta != nullptr || p.decay_tok != 0 || p.z == nullptr;
+    auto intra = gates ? gdn2_chunk_intra_tc_kernel<true> : gdn2_chunk_intra_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ismem);
     if (e != cudaSuccess) return e;
-    gdn2_chunk_intra_tc_kernel<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);
+    intra<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)ChainSmem::TOTAL + 1024;

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GDELTA_ABI_VERSION 1
+#define GDELTA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GDELTA_API __attribute__((visibility("default")))
@@ -85,6 +85,16 @@ typedef enum gdelta_fwd_path {
  *   q, k, z, b : [B, T, H, d_k]  dtype        query, key, readout logit, erase gate
  *   v, w, g    : [B, T, H, d_v]  dtype        value, write gate, output gate
  *   log_alpha  : [B, T, H, d_k]  fp32, <= 0   log of the per-channel decay
+ *                ([B, T, H] when decay_per_token is 1)
+ *   z          : may be NULL: read as 0, so 2 sigmoid(z) = 1 (no dynamic
+ *                readout gain, the static profile alone)
+ *   beta       : [B, T, H] dtype or NULL.  When given, b and w must be NULL
+ *                and b = w = beta on every channel: the KDA parameterisation,
+ *                and with decay_per_token = 1 the Gated DeltaNet one (ETH study,
+ *                "Gated DeltaNet-2": equal erase and write gates reduce GDN-2
+ *                to KDA, a scalar decay further to Gated DeltaNet; "Kimi3 =
+ *                GPT2 x 22580" §5, §6).  The kernels then read one value per
+ *                token and head instead of two d-long rows.
  *   gamma_stat : [H, d_k]        fp32         static readout profile; NULL = ones
  *   S_in       : [B, H, d_k, d_v] fp32        state before token 0; NULL = zeros
  *   S_out      : [B, H, d_k, d_v] fp32        state after token T-1; NULL = not
@@ -119,6 +129,9 @@ typedef struct gdelta_fwd_args {
     float eps;
     void *workspace;
     size_t workspace_bytes;
+    const void *beta;           /* see above; NULL = per-channel b and w */
+    int32_t decay_per_token;    /* 1: log_alpha is [B, T, H] */
+    int32_t reserved2;          /* must be 0 */
 } gdelta_fwd_args;
 
 /*
@@ -127,7 +140,9 @@ typedef struct gdelta_fwd_args {
  * §1/§3: decoding reads and rewrites the fixed-size cache).
  *
  *   q, k, z, b : [B, H, d_k] dtype;  v, w, g : [B, H, d_v] dtype
- *   log_alpha  : [B, H, d_k] fp32;   gamma_stat : [H, d_k] fp32 or NULL
+ *   log_alpha  : [B, H, d_k] fp32 ([B, H] when decay_per_token is 1)
+ *   gamma_stat : [H, d_k] fp32 or NULL
+ *   z may be NULL; beta ([B, H] dtype) replaces b and w as in gdelta_fwd_args
  *   S          : [B, H, d_k, d_v] fp32, read as S_{t-1}, overwritten with S_t
  *   y          : [B, H, d_v] dtype;  o_raw : [B, H, d_v] fp32 or NULL
  */
@@ -143,6 +158,9 @@ typedef struct gdelta_decode_args {
     void *y;
     float *o_raw;
     float eps;
+    const void *beta;           /* NULL = per-channel b and w */
+    int32_t decay_per_token;    /* 1: log_alpha is [B, H] */
+    int32_t reserved2;          /* must be 0 */
 } gdelta_decode_args;
 
 /* ABI version of the loaded library (GDELTA_ABI_VERSION it was built with). */

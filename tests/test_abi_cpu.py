@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.gdelta_abi_version() == 1
+    assert lib.gdelta_abi_version() == 2
     for code in range(8):
         s = lib.gdelta_status_string(code)
         assert s and s != b"unknown status"
@@ -77,6 +77,39 @@ def test_host_validation_codes(lib):
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # null tensors
     d.reserved = 3
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
+
+
+def test_reduced_gate_forms_are_validated_on_the_host(lib):
+    f = lib.gdelta_fwd_chunked
+    beta = 0x20000
+    # beta stands for b and w: giving it beside either is ambiguous
+    assert f(ctypes.byref(_args(beta=beta)), None) == 1
+    assert f(ctypes.byref(_args(beta=beta, b=None)), None) == 1
+    assert f(ctypes.byref(_args(beta=beta, w=None)), None) == 1
+    # without beta both per-channel gates are needed
+    assert f(ctypes.byref(_args(b=None)), None) == 1
+    assert f(ctypes.byref(_args(w=None)), None) == 1
+    assert f(ctypes.byref(_args(decay_per_token=2)), None) == 1
+    assert f(ctypes.byref(_args(reserved2=1)), None) == 1
+    assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(beta=beta))) == -1
+    # accepted forms: no z; beta alone; beta with a per-token decay
+    for kw in ({"z": None}, {"b": None, "w": None, "beta": beta},
+               {"b": None, "w": None, "beta": beta, "decay_per_token": 1, "z": None}):
+        assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(**kw))) in (1, 2), kw
+        assert lib.gdelta_fwd_workspace_bytes(ctypes.byref(_args(**kw))) >= 0
+    d = _native.DecodeArgs()
+    d.B, d.H, d.dk, d.dv, d.dtype = 1, 1, 128, 128, 1
+    for i, n in enumerate(("q", "k", "b", "v", "w", "g", "log_alpha", "S", "y")):
+        setattr(d, n, 0x10000 + 256 * i)
+    d.eps = 1e-6
+    d.beta = beta
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # beta beside b and w
+    d.beta, d.reserved2 = None, 1
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
+    d.reserved2, d.decay_per_token = 0, 5
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
+    d.decay_per_token, d.b = 0, None
+    assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # b missing, no beta
 
 
 def test_path_selection_is_host_logic(lib):

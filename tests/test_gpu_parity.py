@@ -281,3 +281,106 @@ def test_tc_rejects_unsupported_shapes():
         gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], path="tc")
     assert gd.gdelta_fwd_selected_path(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
                                        d["log_alpha"]) == "simt"
+
+
+# --------------------------------------------------------------------------
+# Reduced gate forms: no z, one beta for b and w (KDA), and a per-token decay
+# on top (Gated DeltaNet).  The kernels read the reduced tensors; the oracle
+# gets the same values broadcast over the channels, with z = 0.
+# --------------------------------------------------------------------------
+
+FORMS = {
+    "no_z": dict(drop_z=True, beta=False, decay_tok=False),
+    "kda": dict(drop_z=False, beta=True, decay_tok=False),
+    "gdn": dict(drop_z=True, beta=True, decay_tok=True),
+}
+
+
+def _reduce(inp, form):
+    """(kernel inputs, oracle inputs) for one gate form.  beta is channel 0 of
+    w (a sigmoid, as a write strength is); the per-token log-decay is channel 0
+    of log_alpha."""
+    f = FORMS[form]
+    ker, ref = dict(inp), dict(inp)
+    dk, dv = inp["k"].shape[-1], inp["v"].shape[-1]
+    if f["drop_z"]:
+        ker["z"] = None
+        ref["z"] = torch.zeros_like(inp["z"])
+    if f["beta"]:
+        beta = inp["w"][..., 0].contiguous()
+        ker["beta"], ker["b"], ker["w"] = beta, None, None
+        ref["b"] = beta[..., None].expand(*beta.shape, dk).contiguous()
+        ref["w"] = beta[..., None].expand(*beta.shape, dv).contiguous()
+    if f["decay_tok"]:
+        la = inp["log_alpha"][..., 0].contiguous()
+        ker["log_alpha"] = la
+        ref["log_alpha"] = la[..., None].expand(*la.shape, dk).contiguous()
+    return ker, ref, f["decay_tok"]
+
+
+def _fwd_reduced(ker, decay_tok, **kw):
+    import channel_gated_delta_b200 as gd
+    d = to_dev(ker)
+    B, T, H, dk = d["q"].shape
+    o_raw = torch.empty((B, T, H, d["v"].shape[-1]), dtype=torch.float32, device="cuda")
+    y, S = gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d.get("b"), d.get("w"), d.get("z"), d["g"],
+                                 d["log_alpha"], gamma_stat=d["gamma_stat"], o_raw=o_raw,
+                                 beta=d.get("beta"), decay_per_token=decay_tok, **kw)
+    torch.cuda.synchronize()
+    assert gd.gdelta_get_last_device_error() == 0
+    return y.cpu(), S.cpu(), o_raw.cpu()
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_reduced_gate_forms_bf16(form, path):
+    shape = synth.GdnShape(B=2, T=64 * 3 + 29, H=2, dk=128, dv=128, dtype="bf16", hot_channels=6,
+                           seed=61)
+    ker, ref_in, tok = _reduce(synth.generate(shape), form)
+    y, S, o = _fwd_reduced(ker, tok, path=path)
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, _ref(ref_in, heads), heads, TOL_BF16)
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+def test_reduced_gate_forms_f32(form):
+    shape = synth.GdnShape(B=1, T=101, H=2, dk=64, dv=128, dtype="f32", seed=62)
+    ker, ref_in, tok = _reduce(synth.generate(shape), form)
+    y, S, o = _fwd_reduced(ker, tok, path="simt", chunk=32)
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, _ref(ref_in, heads), heads, TOL_F32)
+
+
+def test_tc_per_token_decay_with_shortened_windows():
+    """A scalar decay fast enough that some 64-token windows exceed the fp16
+    span budget: the chain's own shortened chunks read the per-token decay
+    and the single beta too."""
+    shape = synth.GdnShape(B=1, T=64 * 5 + 3, H=2, dk=128, dv=128, dtype="bf16", seed=63)
+    ker, ref_in, tok = _reduce(synth.generate(shape), "gdn")
+    for side in (ker, ref_in):
+        la = side["log_alpha"].clone()
+        la[:, 64:128] *= 40.0
+        la[:, 256:] *= 40.0
+        side["log_alpha"] = la
+    y, S, o = _fwd_reduced(ker, tok, path="tc")
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, _ref(ref_in, heads), heads, TOL_BF16)
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+def test_decode_reduced_gate_forms(form):
+    import channel_gated_delta_b200 as gd
+    B, H, dk, dv, steps = 3, 2, 128, 128, 4
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(5)) * 0.3
+    S = S0.cuda()
+    heads = oracle.all_heads(B, H)
+    Sref = S0.reshape(B * H, dk, dv).double().numpy()
+    for s in range(steps):
+        ker, ref_in, tok = _reduce(synth.decode_step_inputs(s, seed=71, B=B, H=H, dk=dk, dv=dv), form)
+        d = to_dev(ker)
+        y = gd.gdelta_decode_step(d["q"], d["k"], d["v"], d.get("b"), d.get("w"), d.get("z"), d["g"],
+                                  d["log_alpha"], S, beta=d.get("beta"), decay_per_token=tok)
+        ref = oracle.decode_steps([ref_in], Sref, heads=heads)
+        Sref = ref["S"]
+        assert err_stored(y.cpu().reshape(B * H, dv), ref["y"][0], "bf16") <= TOL_BF16
+    assert err(S.cpu().reshape(B * H, dk, dv), Sref) <= TOL_BF16
