@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stream-tokens", type=int, default=0,
+                    help="also serve one long stream (B1 H16) of this many tokens: forward calls of "
+                         "16384 tokens carrying the state, then decode steps (0 = off)")
     ap.add_argument("--no-forms", action="store_true",
                     help="skip the forward timings of the reduced gate forms")
     # profiling aid: a smaller case of the same workload (fewer batch rows) for
@@ -283,6 +286,9 @@ def run_ours(args, rank, local, world):
     # ---- forward alone on the reduced gate forms (same workload shape)
     forms = None if args.no_forms else run_forms(args, gd, d, shape, dev, stream, ws, world)
 
+    # ---- one long stream: consecutive forward calls, then decode (opt-in)
+    stream_res = run_stream(args, gd, d, shape, dev, stream, world) if args.stream_tokens > 0 else None
+
     # ---- end to end through the public API with host buffers
     e2e = None if args.no_e2e else run_e2e(args, gd, host, dev, stream, shape, world, path)
 
@@ -336,6 +342,7 @@ def run_ours(args, rank, local, world):
         "clocks": clk,
         "decode": dec,
         "forms": forms,
+        "stream": stream_res,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -446,6 +453,66 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
         out[name] = {"fwd_ms_median": ms, "tokens_per_s": B * T * world / (ms * 1e-3),
                      "algorithmic_bytes": nb, "achieved_gbs": gbs, "frac": gbs / hbm, "timed_calls": n}
     return out
+
+
+def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):
+    """One sequence served for ``args.stream_tokens`` tokens: the workload's
+    [B,T,H,d] tensors read as one [1, B*T, H, d] segment (B-major layout makes
+    that a view), forward calls over that segment repeated with the state
+    carried in place, then single-token decode steps on the same state."""
+    import synth
+    B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+    seg = B * T
+    v1 = {k: (t.view(1, seg, H, t.shape[-1]) if t.dim() == 4 else t) for k, t in d.items()}
+    S = torch.zeros(1, H, dk, dv, device=dev)
+    y = torch.empty(1, seg, H, dv, dtype=torch.bfloat16, device=dev)
+    ws_bytes = gd.gdelta_fwd_workspace_bytes(v1["q"], v1["k"], v1["v"], v1["b"], v1["w"], v1["z"], v1["g"],
+                                             v1["log_alpha"], chunk=C, path=args.path)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    n_calls = max(1, -(-args.stream_tokens // seg))
+    dec = [{k: t.to(dev) for k, t in synth.decode_step_inputs(i, seed=91, B=1, H=H, dk=dk, dv=dv).items()}
+           for i in range(4)]
+    y1 = torch.empty(1, H, dv, dtype=torch.bfloat16, device=dev)
+
+    def call():
+        gd.gdelta_fwd_chunked(v1["q"], v1["k"], v1["v"], v1["b"], v1["w"], v1["z"], v1["g"], v1["log_alpha"],
+                              gamma_stat=d["gamma_stat"], S_in=S, S_out=S, y=y, chunk=C, path=args.path,
+                              workspace=ws, stream=stream)
+
+    def step(i):
+        t = dec[i % len(dec)]
+        gd.gdelta_decode_step(t["q"], t["k"], t["v"], t["b"], t["w"], t["z"], t["g"], t["log_alpha"], S,
+                              gamma_stat=d["gamma_stat"], y=y1, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    S.zero_()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    barrier(world)
+    ev[0].record(stream)
+    for _ in range(n_calls):
+        call()
+    ev[1].record(stream)
+    for i in range(decode_steps):
+        step(i)
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    if gd.gdelta_get_last_device_error(stream) != 0:
+        raise RuntimeError("device status word set during the stream")
+    pre_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world)
+    dec_ms = max_over_ranks(ev[1].elapsed_time(ev[2]), world)
+    return {
+        "workload": f"one stream per GPU, B1 H{H} dk=dv={dk}: {n_calls * seg} tokens in {n_calls} forward calls "
+                    f"of {seg} tokens (the workload's tensors read as one sequence, repeated), state carried "
+                    f"in place, then {decode_steps} decode steps",
+        "tokens": n_calls * seg,
+        "prefill_tokens_per_s": n_calls * seg * world / (pre_ms * 1e-3),
+        "prefill_ms_per_call": pre_ms / n_calls,
+        "decode_us_per_step": dec_ms * 1e3 / decode_steps,
+        "state_bytes": H * dk * dv * 4,
+        "finite": bool(torch.isfinite(S).all().item()),
+    }
 
 
 def run_e2e(args, gd, host, dev, stream, shape, world, path):

@@ -1020,9 +1020,10 @@ constexpr uint32_t kItmW = 0;      // W' (M=64) reuses the columns of P after it
 constexpr uint32_t kItmN = 128;    // N  (M=64)
 }  // namespace
 
-// kGates: the gate inputs may come in their reduced forms (one beta for b and w,
-// one log-decay per token, no z); false compiles the plain per-channel loads.
-template <bool kGates>
+// Gate forms, fixed at compile time: kNoZ reads no z (2 sigmoid(z) = 1), kBeta
+// reads one beta per token and head for both b and w, kTok one log-decay per
+// token and head.  All false is the per-channel GDN-2 form.
+template <bool kNoZ, bool kBeta, bool kTok>
 __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
     using L = IntraSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1089,7 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gk = gt * kDK + c4;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (in) {
-                if (kGates && p.decay_tok) {
+                if (kTok) {
                     const float s = __ldg(p.la + gt);
                     x = make_float4(s, s, s, s);
                 } else {
@@ -1099,9 +1100,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             la[u][0] = x.x * kLog2e; la[u][1] = x.y * kLog2e; la[u][2] = x.z * kLog2e; la[u][3] = x.w * kLog2e;
             kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
             kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-            kq[u][2] = in && (!kGates || p.z) ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+            kq[u][2] = in && !kNoZ ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
             kq[u][3] = !in ? make_uint2(0, 0)
-                      : kGates && p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
+                      : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
         }
 #pragma unroll
         for (int u = 1; u < 8; ++u)
@@ -1228,7 +1229,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gv = gt * kDV + c4;
             vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
             vw[u][1] = !in ? make_uint2(0, 0)
-                      : kGates && p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                      : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
         }
         tc::fence_proxy_async();
         __syncthreads();
@@ -1437,8 +1438,13 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.wflags = wflags;
 
     const size_t ismem = (size_t)IntraSmem::TOTAL + 1024;
-    const bool gates = p.beta != nullptr || p.decay_tok != 0 || p.z == nullptr;
-    auto intra = gates ? gdn2_chunk_intra_tc_kernel<true> : gdn2_chunk_intra_tc_kernel<false>;
+    using IntraFn = void (*)(TcParams, uint8_t *, int *);
+    static constexpr IntraFn kIntra[8] = {
+        gdn2_chunk_intra_tc_kernel<false, false, false>, gdn2_chunk_intra_tc_kernel<false, false, true>,
+        gdn2_chunk_intra_tc_kernel<false, true, false>,  gdn2_chunk_intra_tc_kernel<false, true, true>,
+        gdn2_chunk_intra_tc_kernel<true, false, false>,  gdn2_chunk_intra_tc_kernel<true, false, true>,
+        gdn2_chunk_intra_tc_kernel<true, true, false>,   gdn2_chunk_intra_tc_kernel<true, true, true>};
+    const IntraFn intra = kIntra[(p.z == nullptr) * 4 + (p.beta != nullptr) * 2 + (p.decay_tok != 0)];
     cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ismem);
     if (e != cudaSuccess) return e;
     intra<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);

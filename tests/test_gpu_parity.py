@@ -384,3 +384,50 @@ def test_decode_reduced_gate_forms(form):
         Sref = ref["S"]
         assert err_stored(y.cpu().reshape(B * H, dv), ref["y"][0], "bf16") <= TOL_BF16
     assert err(S.cpu().reshape(B * H, dk, dv), Sref) <= TOL_BF16
+
+
+# --------------------------------------------------------------------------
+# Long streams: prefill in consecutive calls carrying the state, then decode
+# (Muir review §4.3: one continuous token stream far beyond the training
+# length, served with a fixed-size fp32 state).
+# --------------------------------------------------------------------------
+
+def test_long_stream_prefill_calls_then_decode():
+    """131072 tokens of one sequence (B1, two heads) in 8 forward calls of
+    16384 tokens on the tensor-core path, the state updated in place between
+    calls, then 16 decode steps.  Every output of every call and the final
+    state are compared with the oracle run over the same stream, so error
+    that accumulated across 2048 windows of state carries would show."""
+    import channel_gated_delta_b200 as gd
+    seg, n_seg, H = 16384, 8, 2
+    S = torch.zeros(1, H, 128, 128, device="cuda")
+    heads = oracle.all_heads(1, H)
+    Sref = np.zeros((H, 128, 128))
+    gamma = None
+    worst = 0.0
+    for i in range(n_seg):
+        shape = synth.GdnShape(B=1, T=seg, H=H, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=200 + i)
+        inp = synth.generate(shape)
+        if gamma is None:
+            gamma = inp["gamma_stat"]
+        inp["gamma_stat"] = gamma                       # one layer: the same static profile throughout
+        d = to_dev(inp)
+        y, _ = gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"],
+                                     gamma_stat=d["gamma_stat"], S_in=S, S_out=S, path="tc")
+        torch.cuda.synchronize()
+        assert gd.gdelta_get_last_device_error() == 0
+        ref = _ref(inp, heads, S0=Sref)
+        Sref = ref["S"]
+        worst = max(worst, err_stored(sel_heads(y.cpu(), heads), ref["y"], "bf16"))
+    assert worst <= TOL_BF16, worst
+    assert err(S.cpu().reshape(H, 128, 128), Sref) <= TOL_BF16
+    gam = gamma.cuda()
+    for s in range(16):
+        inp = synth.decode_step_inputs(s, seed=81, B=1, H=H, dk=128, dv=128)
+        d = to_dev(inp)
+        y = gd.gdelta_decode_step(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                  d["log_alpha"], S, gamma_stat=gam)
+        ref = oracle.decode_steps([inp], Sref, gamma_stat=gamma, heads=heads)
+        Sref = ref["S"]
+        assert err_stored(y.cpu().reshape(H, 128), ref["y"][0], "bf16") <= TOL_BF16
+    assert err(S.cpu().reshape(H, 128, 128), Sref) <= TOL_BF16
