@@ -502,6 +502,22 @@ def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):
         raise RuntimeError("device status word set during the stream")
     pre_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world)
     dec_ms = max_over_ranks(ev[1].elapsed_time(ev[2]), world)
+
+    # the pieces a rank of a sequence-sharded forward adds: the segment map
+    # (two forward calls) and one affine composition of the state
+    A, D = gd.gdelta_segment_map(v1["q"], v1["k"], v1["v"], v1["b"], v1["w"], v1["z"], v1["g"], v1["log_alpha"],
+                                 chunk=C, path=args.path, stream=stream)
+    S2 = torch.empty_like(S)
+    sm = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    sm[0].record(stream)
+    gd.gdelta_segment_map(v1["q"], v1["k"], v1["v"], v1["b"], v1["w"], v1["z"], v1["g"], v1["log_alpha"],
+                          chunk=C, path=args.path, stream=stream)
+    sm[1].record(stream)
+    gd.gdelta_state_affine(A, S_in=S, D=D, S_out=S2, stream=stream)
+    sm[2].record(stream)
+    torch.cuda.synchronize(dev)
+    map_ms = max_over_ranks(sm[0].elapsed_time(sm[1]), world)
+    aff_ms = max_over_ranks(sm[1].elapsed_time(sm[2]), world)
     return {
         "workload": f"one stream per GPU, B1 H{H} dk=dv={dk}: {n_calls * seg} tokens in {n_calls} forward calls "
                     f"of {seg} tokens (the workload's tensors read as one sequence, repeated), state carried "
@@ -510,6 +526,8 @@ def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):
         "prefill_tokens_per_s": n_calls * seg * world / (pre_ms * 1e-3),
         "prefill_ms_per_call": pre_ms / n_calls,
         "decode_us_per_step": dec_ms * 1e3 / decode_steps,
+        "segment_map_ms": map_ms,
+        "state_affine_us": aff_ms * 1e3,
         "state_bytes": H * dk * dv * 4,
         "finite": bool(torch.isfinite(S).all().item()),
     }

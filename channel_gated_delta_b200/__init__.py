@@ -30,6 +30,8 @@ __all__ = [
     "gdelta_fwd_workspace_bytes",
     "gdelta_fwd_selected_path",
     "gdelta_state_init",
+    "gdelta_state_affine",
+    "gdelta_segment_map",
     "gdelta_fwd_chunked",
     "gdelta_decode_step",
     "gdelta_get_last_device_error",
@@ -151,6 +153,54 @@ def gdelta_state_init(S: torch.Tensor, S_src: Optional[torch.Tensor] = None, str
     ps = _dev_ptr(S_src, "S_src", torch.float32, tuple(S.shape), required=False)
     _check(_lib().gdelta_state_init(p, B, H, dk, dv, ps, _stream(stream)), "gdelta_state_init")
     return S
+
+
+def gdelta_state_affine(A: torch.Tensor, S_in: Optional[torch.Tensor] = None, D: Optional[torch.Tensor] = None,
+                        S_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """S_out = A S_in + D per (batch, head).  A [B,H,dk,dk], S_in / D / S_out
+    [B,H,dk,dv] fp32 on the GPU; S_in or D None reads as zero; S_out may be D.
+    Returns S_out (allocated when not given)."""
+    if A.dim() != 4 or A.shape[-1] != A.shape[-2]:
+        raise ValueError("A must be [B, H, dk, dk]")
+    B, H, dk, _ = A.shape
+    ref = S_in if S_in is not None else D if D is not None else S_out
+    if ref is None:
+        raise ValueError("one of S_in, D, S_out is needed for d_v")
+    dv = ref.shape[-1]
+    shp = (B, H, dk, dv)
+    if S_out is None:
+        S_out = torch.empty(shp, dtype=torch.float32, device=A.device)
+    _check(_lib().gdelta_state_affine(_dev_ptr(S_out, "S_out", torch.float32, shp),
+                                      _dev_ptr(A, "A", torch.float32, (B, H, dk, dk)),
+                                      _dev_ptr(S_in, "S_in", torch.float32, shp, required=False),
+                                      _dev_ptr(D, "D", torch.float32, shp, required=False),
+                                      B, H, dk, dv, _stream(stream)), "gdelta_state_affine")
+    return S_out
+
+
+def gdelta_segment_map(q, k, v, b, w, z, g, log_alpha, *, beta=None, decay_per_token: bool = False,
+                       chunk: int = 64, path: str = "auto", stream=None
+                       ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(A, D) with S_end = A S_start + D for this segment of tokens, every
+    (batch, head): A [B,H,dk,dk] is the forward's final state from S_in = I
+    with zero values (d_v = d_k), D its final state from S_in = 0.  Two
+    forward calls; their y is scratch.  z does not reach the state and is not
+    read (g is read only for the scratch y)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    zeros = torch.zeros((B, T, H, dk), dtype=q.dtype, device=dev)     # v, w and g of the A pass
+    eye = torch.eye(dk, dtype=torch.float32, device=dev).expand(B, H, dk, dk).contiguous()
+    A = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    D = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    y_a = torch.empty((B, T, H, dk), dtype=q.dtype, device=dev)
+    y_d = y_a if dv == dk else torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    gdelta_fwd_chunked(q, k, zeros, b, None if beta is not None else zeros, None, zeros, log_alpha,
+                       S_in=eye, S_out=A, y=y_a, chunk=chunk, path=path, stream=stream, beta=beta,
+                       decay_per_token=decay_per_token)
+    gdelta_fwd_chunked(q, k, v, b, w, None, g, log_alpha, S_out=D, y=y_d, chunk=chunk, path=path,
+                       stream=stream, beta=beta, decay_per_token=decay_per_token)
+    return A, D
 
 
 def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=None, S_out=None,

@@ -33,6 +33,7 @@ EXPORTED = (
     "gdelta_fwd_workspace_bytes",
     "gdelta_fwd_selected_path",
     "gdelta_state_init",
+    "gdelta_state_affine",
     "gdelta_fwd_chunked",
     "gdelta_fwd_chunked_noalloc",
     "gdelta_decode_step",
@@ -92,6 +93,9 @@ def load(path: str = LIB_PATH):
     lib.gdelta_state_init.restype = ctypes.c_int
     lib.gdelta_state_init.argtypes = [_fp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_int32, _fp, _vp]
+    lib.gdelta_state_affine.restype = ctypes.c_int
+    lib.gdelta_state_affine.argtypes = [_fp, _fp, _fp, _fp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, _vp]
     lib.gdelta_fwd_chunked.restype = ctypes.c_int
     lib.gdelta_fwd_chunked.argtypes = [ctypes.POINTER(FwdArgs), _vp]
     lib.gdelta_fwd_chunked_noalloc.restype = ctypes.c_int

@@ -65,6 +65,8 @@ cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
 size_t fwd_simt_smem_bytes(int dk, int dv, int C);
 int fwd_simt_chunk(int dk, int dv, int requested);
 cudaError_t launch_state_init(float *S, const float *src, size_t n, cudaStream_t stream);
+cudaError_t launch_state_affine(float *S_out, const float *A, const float *S_in, const float *D, int BH, int dk,
+                                int dv, cudaStream_t stream);
 cudaError_t launch_fwd_tc(const FwdParams &p, void *workspace, cudaStream_t stream);
 size_t fwd_tc_workspace_bytes(int B, int H, int T);
 bool fwd_tc_supported(int dtype, int dk, int dv, int chunk);

@@ -106,6 +106,25 @@ gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32_t dk, int3
                                                                                : GDELTA_ERR_CUDA;
 }
 
+static bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b) return false;
+    const char *x = (const char *)a, *y = (const char *)b;
+    return x < y + nb && y < x + na;
+}
+
+gdelta_status gdelta_state_affine(float *S_out, const float *A, const float *S_in, const float *D, int32_t B,
+                                  int32_t H, int32_t dk, int32_t dv, void *stream) {
+    if (!S_out || !A || B < 1 || H < 1) return GDELTA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDELTA_ERR_UNSUPPORTED;
+    if (!aligned16(S_out) || !aligned16(A) || !aligned16(S_in) || !aligned16(D)) return GDELTA_ERR_ALIGNMENT;
+    const size_t ns = (size_t)B * H * dk * dv * sizeof(float), na = (size_t)B * H * dk * dk * sizeof(float);
+    if (overlaps(S_out, ns, A, na) || overlaps(S_out, ns, S_in, ns)) return GDELTA_ERR_INVALID_ARG;
+    if (D && D != S_out && overlaps(S_out, ns, D, ns)) return GDELTA_ERR_INVALID_ARG;
+    return launch_state_affine(S_out, A, S_in, D, B * H, dk, dv, (cudaStream_t)stream) == cudaSuccess
+               ? GDELTA_OK
+               : GDELTA_ERR_CUDA;
+}
+
 gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     gdelta_status st = check_fwd(a);
     if (st != GDELTA_OK) return st;

@@ -186,6 +186,26 @@ GDELTA_API int gdelta_fwd_selected_path(const gdelta_fwd_args *args);
 GDELTA_API gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32_t dk, int32_t dv,
                                 const float *S_src, void *stream);
 
+/*
+ * Affine state map: S_out = A S_in + D for every (batch, head).
+ *   A           : [B, H, d_k, d_k] fp32   the map's linear part
+ *   S_in, D     : [B, H, d_k, d_v] fp32   either may be NULL (read as 0)
+ *   S_out       : [B, H, d_k, d_v] fp32   written; may be D itself, must not
+ *                 overlap A or S_in (GDELTA_ERR_INVALID_ARG otherwise)
+ * Every token's update is affine in the state with a linear part that acts
+ * on the key rows and is the same for every value column, so a whole segment
+ * of tokens moves the state by S_end = A S_start + D ("Kimi3 = GPT2 x 22580"
+ * §4: a chunk's transition is the product of its tokens' generalised
+ * Householder factors plus an accumulated write; §5 and §6 add the decays).
+ * A is what gdelta_fwd_chunked returns as S_out from S_in = I with v = 0 (and
+ * d_v = d_k); D is its S_out from S_in = 0.  Composing the maps of
+ * consecutive segments gives each segment its starting state without running
+ * the segments one after another (a long sequence split over devices).
+ * Asynchronous on `stream`.
+ */
+GDELTA_API gdelta_status gdelta_state_affine(float *S_out, const float *A, const float *S_in, const float *D,
+                                             int32_t B, int32_t H, int32_t dk, int32_t dv, void *stream);
+
 /* Chunked forward; see gdelta_fwd_args. */
 GDELTA_API gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *args, void *stream);
 

@@ -112,6 +112,20 @@ def test_reduced_gate_forms_are_validated_on_the_host(lib):
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # b missing, no beta
 
 
+def test_state_affine_validation(lib):
+    f = lib.gdelta_state_affine
+    S, A, S_in, D = 0x100000, 0x200000, 0x300000, 0x400000
+    n = 128 * 128 * 4
+    assert f(None, A, S_in, D, 1, 1, 128, 128, None) == 1
+    assert f(S, None, S_in, D, 1, 1, 128, 128, None) == 1
+    assert f(S, A, S_in, D, 0, 1, 128, 128, None) == 1
+    assert f(S, A, S_in, D, 1, 1, 96, 128, None) == 2
+    assert f(S, A + 4, S_in, D, 1, 1, 128, 128, None) == 3
+    assert f(S, A, S + n // 2, D, 1, 1, 128, 128, None) == 1        # S_in overlaps S_out
+    assert f(S, S + 16, S_in, D, 1, 1, 128, 128, None) == 1          # A overlaps S_out
+    assert f(S, A, S_in, S + 16, 1, 1, 128, 128, None) == 1          # D partly over S_out
+
+
 def test_path_selection_is_host_logic(lib):
     a = _args()
     assert lib.gdelta_fwd_selected_path(ctypes.byref(a)) in (1, 2)

@@ -431,3 +431,60 @@ def test_long_stream_prefill_calls_then_decode():
         Sref = ref["S"]
         assert err_stored(y.cpu().reshape(H, 128), ref["y"][0], "bf16") <= TOL_BF16
     assert err(S.cpu().reshape(H, 128, 128), Sref) <= TOL_BF16
+
+
+# --------------------------------------------------------------------------
+# Sequence sharding: segment maps, their composition, and the forward from
+# the composed state, with the segments run one after another on this GPU
+# exactly as separate ranks would run them.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64), (64, 64)])
+def test_state_affine_matches_float64(dk, dv):
+    import channel_gated_delta_b200 as gd
+    gen = torch.Generator().manual_seed(dk + dv)
+    B, H = 2, 3
+    A = torch.randn(B, H, dk, dk, generator=gen) / dk ** 0.5
+    S = torch.randn(B, H, dk, dv, generator=gen)
+    D = torch.randn(B, H, dk, dv, generator=gen)
+    ref = (A.double() @ S.double() + D.double()).numpy()
+    Ad, Sd, Dd = A.cuda(), S.cuda(), D.cuda()
+    assert err(gd.gdelta_state_affine(Ad, S_in=Sd, D=Dd), ref) <= TOL_F32
+    assert err(gd.gdelta_state_affine(Ad, S_in=Sd), (A.double() @ S.double()).numpy()) <= TOL_F32
+    assert torch.equal(gd.gdelta_state_affine(Ad, D=Dd).cpu(), D)          # zero state: D itself
+    gd.gdelta_state_affine(Ad, S_in=Sd, D=Dd, S_out=Dd)                     # in place on D
+    torch.cuda.synchronize()
+    assert err(Dd, ref) <= TOL_F32
+    with pytest.raises(gd.GdeltaError):
+        gd.gdelta_state_affine(Ad, S_in=Sd, S_out=Sd)                        # output over the input
+
+
+@pytest.mark.parametrize("dtype,path,dk,dv", [("bf16", "tc", 128, 128), ("f32", "simt", 64, 128)])
+def test_seqshard_segments_compose_to_the_whole_sequence(dtype, path, dk, dv):
+    import channel_gated_delta_b200 as gd
+    from channel_gated_delta_b200.seqshard import compose_affine, compose_range
+    n_seg, H = 4, 2
+    bounds = [0, 150, 301, 470, 637]                   # ragged: windows cross segment ends
+    inp = synth.generate(synth.GdnShape(B=1, T=bounds[-1], H=H, dk=dk, dv=dv, dtype=dtype,
+                                        hot_channels=6 if dtype == "bf16" else 0, seed=93))
+    d = to_dev(inp)
+    segs = [{k: (v[:, bounds[r]:bounds[r + 1]] if v.dim() == 4 else v) for k, v in d.items()}
+            for r in range(n_seg)]
+    maps = [gd.gdelta_segment_map(s["q"], s["k"], s["v"], s["b"], s["w"], s["z"], s["g"], s["log_alpha"],
+                                  path=path) for s in segs]
+    As, Ds = [m[0] for m in maps], [m[1] for m in maps]
+    ys, finals = [], []
+    for r, s in enumerate(segs):
+        S0 = compose_range(As, Ds, 0, r, None, compose_affine)
+        y, S_end = gd.gdelta_fwd_chunked(s["q"], s["k"], s["v"], s["b"], s["w"], s["z"], s["g"], s["log_alpha"],
+                                         gamma_stat=d["gamma_stat"], S_in=S0, path=path)
+        ys.append(y)
+        finals.append(compose_range(As, Ds, r + 1, n_seg, S_end, compose_affine))
+    torch.cuda.synchronize()
+    assert gd.gdelta_get_last_device_error() == 0
+    heads = oracle.all_heads(1, H)
+    ref = _ref(inp, heads)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    assert err_stored(sel_heads(torch.cat(ys, 1).cpu(), heads), ref["y"], dtype) <= tol
+    for S_fin in finals:                              # every rank ends with the sequence's final state
+        assert err(S_fin.cpu().reshape(H, dk, dv), ref["S"]) <= tol
