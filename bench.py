@@ -409,6 +409,8 @@ FORMS = {
     "kda": dict(z=True, beta=True, decay_tok=False),
     # Gated DeltaNet: one beta and one scalar decay per token, no z
     "gdn": dict(z=False, beta=True, decay_tok=True),
+    # per-channel gates on pre-activation q and k: SiLU and l2 norm in the kernels
+    "raw_qk": dict(z=True, beta=False, decay_tok=False, qk_raw=True),
 }
 
 
@@ -426,11 +428,12 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
         beta = d["w"][..., 0].contiguous() if f["beta"] else None
         b, w = (None, None) if f["beta"] else (d["b"], d["w"])
         la = d["log_alpha"][..., 0].contiguous() if f["decay_tok"] else d["log_alpha"]
+        raw = f.get("qk_raw", False)
 
         def call():
             gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], b, w, z, d["g"], la, gamma_stat=d["gamma_stat"],
                                   S_in=S, S_out=S, y=y, chunk=C, path=args.path, workspace=ws,
-                                  stream=stream, beta=beta, decay_per_token=f["decay_tok"])
+                                  stream=stream, beta=beta, decay_per_token=f["decay_tok"], qk_raw=raw)
 
         for _ in range(3):
             gd.gdelta_state_init(S, stream=stream)
@@ -448,10 +451,29 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
             evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
         ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
-        nb = fwd_bytes(B, T, H, dk, dv, 2, **f)
+        nb = fwd_bytes(B, T, H, dk, dv, 2, z=f["z"], beta=f["beta"], decay_tok=f["decay_tok"])
         gbs = nb / (ms * 1e-3) / 1e9
         out[name] = {"fwd_ms_median": ms, "tokens_per_s": B * T * world / (ms * 1e-3),
                      "algorithmic_bytes": nb, "achieved_gbs": gbs, "frac": gbs / hbm, "timed_calls": n}
+        if raw:
+            # for comparison: the same preprocessing as separate PyTorch ops, then the plain forward
+            import torch.nn.functional as F
+            qn = torch.empty_like(d["q"])
+            kn = torch.empty_like(d["k"])
+            ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            for i in range(n):
+                gd.gdelta_state_init(S, stream=stream)
+                ev2[i][0].record(stream)
+                with torch.cuda.stream(stream):
+                    qn.copy_(F.normalize(F.silu(d["q"].float()), dim=-1))
+                    kn.copy_(F.normalize(F.silu(d["k"].float()), dim=-1))
+                gd.gdelta_fwd_chunked(qn, kn, d["v"], b, w, z, d["g"], la, gamma_stat=d["gamma_stat"],
+                                      S_in=S, S_out=S, y=y, chunk=C, path=args.path, workspace=ws,
+                                      stream=stream)
+                ev2[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            out[name]["torch_preprocess_then_fwd_ms_median"] = max_over_ranks(
+                statistics.median(a.elapsed_time(c) for a, c in ev2), world)
     return out
 
 

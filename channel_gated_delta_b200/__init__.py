@@ -95,7 +95,7 @@ def gdelta_status_string(status: int) -> str:
 
 
 def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
-                path, workspace, beta=None, decay_per_token=False) -> _native.FwdArgs:
+                path, workspace, beta=None, decay_per_token=False, qk_raw=False) -> _native.FwdArgs:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -114,6 +114,7 @@ def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_ra
     a.g = _dev_ptr(g, "g", dt, vs)
     a.beta = _dev_ptr(beta, "beta", dt, (B, T, H), required=False)
     a.decay_per_token = int(bool(decay_per_token))
+    a.qk_raw = int(bool(qk_raw))
     a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, (B, T, H) if decay_per_token else ks)
     a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
     a.S_in = _dev_ptr(S_in, "S_in", torch.float32, (B, H, dk, dv), required=False)
@@ -128,16 +129,18 @@ def _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_ra
 
 
 def gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
-                               path: str = "auto", beta=None, decay_per_token: bool = False) -> int:
+                               path: str = "auto", beta=None, decay_per_token: bool = False,
+                               qk_raw: bool = False) -> int:
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
-                    path, None, beta, decay_per_token)
+                    path, None, beta, decay_per_token, qk_raw)
     return int(_lib().gdelta_fwd_workspace_bytes(ctypes.byref(a)))
 
 
 def gdelta_fwd_selected_path(q, k, v, b, w, z, g, log_alpha, *, chunk: int = 64,
-                             path: str = "auto", beta=None, decay_per_token: bool = False) -> str:
+                             path: str = "auto", beta=None, decay_per_token: bool = False,
+                             qk_raw: bool = False) -> str:
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, None, None, None, None, None, chunk, 1e-6,
-                    path, None, beta, decay_per_token)
+                    path, None, beta, decay_per_token, qk_raw)
     code = int(_lib().gdelta_fwd_selected_path(ctypes.byref(a)))
     if code < 0:
         raise GdeltaError(2, "gdelta_fwd_selected_path")
@@ -179,7 +182,7 @@ def gdelta_state_affine(A: torch.Tensor, S_in: Optional[torch.Tensor] = None, D:
 
 
 def gdelta_segment_map(q, k, v, b, w, z, g, log_alpha, *, beta=None, decay_per_token: bool = False,
-                       chunk: int = 64, path: str = "auto", stream=None
+                       qk_raw: bool = False, chunk: int = 64, path: str = "auto", stream=None
                        ) -> Tuple[torch.Tensor, torch.Tensor]:
     """(A, D) with S_end = A S_start + D for this segment of tokens, every
     (batch, head): A [B,H,dk,dk] is the forward's final state from S_in = I
@@ -197,16 +200,16 @@ def gdelta_segment_map(q, k, v, b, w, z, g, log_alpha, *, beta=None, decay_per_t
     y_d = y_a if dv == dk else torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
     gdelta_fwd_chunked(q, k, zeros, b, None if beta is not None else zeros, None, zeros, log_alpha,
                        S_in=eye, S_out=A, y=y_a, chunk=chunk, path=path, stream=stream, beta=beta,
-                       decay_per_token=decay_per_token)
+                       decay_per_token=decay_per_token, qk_raw=qk_raw)
     gdelta_fwd_chunked(q, k, v, b, w, None, g, log_alpha, S_out=D, y=y_d, chunk=chunk, path=path,
-                       stream=stream, beta=beta, decay_per_token=decay_per_token)
+                       stream=stream, beta=beta, decay_per_token=decay_per_token, qk_raw=qk_raw)
     return A, D
 
 
 def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=None, S_out=None,
                        y=None, o_raw=None, chunk: int = 64, eps: float = 1e-6, path: str = "auto",
                        workspace=None, return_state: bool = True, stream=None, beta=None,
-                       decay_per_token: bool = False
+                       decay_per_token: bool = False, qk_raw: bool = False
                        ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked forward over [B,T,H,d] tokens.  Returns (y, S_out).
 
@@ -214,6 +217,8 @@ def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=
     ``beta`` [B,T,H] replaces ``b`` and ``w`` (pass them as None) with one
     gate per token and head; ``decay_per_token`` takes ``log_alpha`` as
     [B,T,H].  Together these give the KDA and Gated DeltaNet special cases.
+    ``qk_raw``: q and k are pre-activation; the kernels apply SiLU and the
+    per-head l2 normalisation as they load them.
 
     Outputs not passed in are allocated with torch on q's device; S_out is
     only allocated when ``return_state``.  ``workspace`` (uint8 CUDA tensor) is
@@ -227,21 +232,21 @@ def gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, *, gamma_stat=None, S_in=
         S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     if workspace is None:
         need = gdelta_fwd_workspace_bytes(q, k, v, b, w, z, g, log_alpha, chunk=chunk, path=path,
-                                          beta=beta, decay_per_token=decay_per_token)
+                                          beta=beta, decay_per_token=decay_per_token, qk_raw=qk_raw)
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     a = _fwd_struct(q, k, v, b, w, z, g, log_alpha, gamma_stat, S_in, S_out, y, o_raw, chunk, eps,
-                    path, workspace, beta, decay_per_token)
+                    path, workspace, beta, decay_per_token, qk_raw)
     _check(_lib().gdelta_fwd_chunked(ctypes.byref(a), _stream(stream)), "gdelta_fwd_chunked")
     return y, S_out
 
 
 def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=None, o_raw=None,
                        eps: float = 1e-6, stream=None, beta=None,
-                       decay_per_token: bool = False) -> torch.Tensor:
+                       decay_per_token: bool = False, qk_raw: bool = False) -> torch.Tensor:
     """One token per (batch, head): S [B,H,dk,dv] fp32 updated in place; returns y [B,H,dv].
 
-    ``z``, ``beta`` and ``decay_per_token`` as in gdelta_fwd_chunked, with
+    ``z``, ``beta``, ``decay_per_token`` and ``qk_raw`` as in gdelta_fwd_chunked, with
     beta [B,H] and a per-token log_alpha [B,H].
     """
     B, H, dk = q.shape
@@ -263,6 +268,7 @@ def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=
     a.g = _dev_ptr(g, "g", dt, vs)
     a.beta = _dev_ptr(beta, "beta", dt, (B, H), required=False)
     a.decay_per_token = int(bool(decay_per_token))
+    a.qk_raw = int(bool(qk_raw))
     a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, (B, H) if decay_per_token else ks)
     a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
     a.S = _dev_ptr(S, "S", torch.float32, (B, H, dk, dv))

@@ -54,7 +54,7 @@ class FwdArgs(ctypes.Structure):
         ("log_alpha", _fp), ("gamma_stat", _fp), ("S_in", _fp), ("S_out", _fp),
         ("y", _vp), ("o_raw", _fp), ("eps", ctypes.c_float),
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
-        ("beta", _vp), ("decay_per_token", ctypes.c_int32), ("reserved2", ctypes.c_int32),
+        ("beta", _vp), ("decay_per_token", ctypes.c_int32), ("qk_raw", ctypes.c_int32),
     ]
 
 
@@ -66,7 +66,7 @@ class DecodeArgs(ctypes.Structure):
         ("v", _vp), ("w", _vp), ("g", _vp),
         ("log_alpha", _fp), ("gamma_stat", _fp), ("S", _fp),
         ("y", _vp), ("o_raw", _fp), ("eps", ctypes.c_float),
-        ("beta", _vp), ("decay_per_token", ctypes.c_int32), ("reserved2", ctypes.c_int32),
+        ("beta", _vp), ("decay_per_token", ctypes.c_int32), ("qk_raw", ctypes.c_int32),
     ]
 
 

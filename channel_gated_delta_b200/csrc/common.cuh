@@ -22,6 +22,16 @@ __device__ __forceinline__ void stf(__nv_bfloat16 *p, size_t i, float x) {
 // 2 * sigmoid(z): the dynamic readout modulation in (0, 2) (Muir review §2.1).
 __device__ __forceinline__ float two_sigmoid(float z) { return 2.0f / (1.0f + expf(-z)); }
 
+// SiLU, x sigmoid(x): the key and query activation before their per-head
+// l2 normalisation (Muir review §2.1).
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+
+// A value as the token dtype holds it (bf16 rounding; fp32 unchanged).
+__device__ __forceinline__ float as_dtype(float x, const float *) { return x; }
+__device__ __forceinline__ float as_dtype(float x, const __nv_bfloat16 *) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -33,7 +43,8 @@ enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2 };
 
 // Gate and decay forms (gdelta.h): z may be null (read as 0); beta, when
 // non-null, replaces b and w (one value per token and head); decay_tok = 1
-// means log_alpha holds one value per token and head.
+// means log_alpha holds one value per token and head; qk_raw = 1 means q and
+// k still need SiLU and per-head l2 normalisation.
 struct FwdParams {
     int B, T, H, dk, dv, C;
     const void *q, *k, *z, *b, *v, *w, *g;
@@ -44,6 +55,7 @@ struct FwdParams {
     float eps;
     const void *beta;
     int decay_tok;
+    int qk_raw;
     int *status;
 };
 
@@ -57,6 +69,7 @@ struct DecodeParams {
     float eps;
     const void *beta;
     int decay_tok;
+    int qk_raw;
 };
 
 // Launchers (return cudaError_t of the launch).

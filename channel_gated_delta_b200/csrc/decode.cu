@@ -22,7 +22,9 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
                  : "memory");
 }
 
-template <typename T, int DK, int DV>
+// kRaw: q and k need SiLU and l2 normalisation (compiled apart, so the plain
+// build keeps its register allocation).
+template <typename T, int DK, int DV, bool kRaw>
 __global__ void __launch_bounds__(256, 4) gdn2_decode_kernel(DecodeParams p) {
     constexpr int NT = 256;
     constexpr int CPR = DV / 4;       // threads across one row (4 columns each)
@@ -63,13 +65,41 @@ __global__ void __launch_bounds__(256, 4) gdn2_decode_kernel(DecodeParams p) {
 
     const T *q = (const T *)p.q, *k = (const T *)p.k, *z = (const T *)p.z, *b = (const T *)p.b;
     const T *v = (const T *)p.v, *w = (const T *)p.w, *beta = (const T *)p.beta;
+    // raw q, k: SiLU, then 1 / ||.|| over the head's d_k channels
+    float inv_k = 1.f, inv_q = 1.f;
+    if (kRaw) {
+        float ssk = 0.f, ssq = 0.f;
+        for (int i = tid; i < DK; i += NT) {
+            const float a = silu(ldf(k, kbase + i)), c = silu(ldf(q, kbase + i));
+            ssk = fmaf(a, a, ssk);
+            ssq = fmaf(c, c, ssq);
+        }
+        ssk = warp_sum(ssk);
+        ssq = warp_sum(ssq);
+        if ((tid & 31) == 0) {
+            s_part[0][tid >> 5] = ssk;
+            s_part[1][tid >> 5] = ssq;
+        }
+        __syncthreads();
+        ssk = 0.f;
+        ssq = 0.f;
+#pragma unroll
+        for (int u = 0; u < NT / 32; ++u) {
+            ssk += s_part[0][u];
+            ssq += s_part[1][u];
+        }
+        inv_k = rsqrtf(fmaxf(ssk, 1e-24f));
+        inv_q = rsqrtf(fmaxf(ssq, 1e-24f));
+        __syncthreads();                              // s_part is reused below
+    }
     float cb = 0.f, ck = 0.f;
     for (int i = tid; i < DK; i += NT) {
-        const float ki = ldf(k, kbase + i);
+        const float ki = kRaw ? as_dtype(silu(ldf(k, kbase + i)) * inv_k, k) : ldf(k, kbase + i);
         const float bi = beta ? ldf(beta, head) : ldf(b, kbase + i);
         const float al = expf(p.decay_tok ? p.la[head] : p.la[kbase + i]);
         const float gs = p.gs ? p.gs[(size_t)h * DK + i] : 1.f;
-        const float qt = ldf(q, kbase + i) * gs * two_sigmoid(z ? ldf(z, kbase + i) : 0.f);
+        const float qi = kRaw ? as_dtype(silu(ldf(q, kbase + i)) * inv_q, q) : ldf(q, kbase + i);
+        const float qt = qi * gs * two_sigmoid(z ? ldf(z, kbase + i) : 0.f);
         s_k[i] = ki;
         s_kh[i] = bi * ki;
         s_alpha[i] = al;
@@ -155,15 +185,20 @@ __global__ void __launch_bounds__(256, 4) gdn2_decode_kernel(DecodeParams p) {
     }
 }
 
-template <typename T>
-static cudaError_t launch_t(const DecodeParams &p, cudaStream_t s) {
+template <typename T, bool kRaw>
+static cudaError_t launch_tr(const DecodeParams &p, cudaStream_t s) {
     const dim3 grid(p.B * p.H), block(256);
-    if (p.dk == 128 && p.dv == 128) gdn2_decode_kernel<T, 128, 128><<<grid, block, 0, s>>>(p);
-    else if (p.dk == 128 && p.dv == 64) gdn2_decode_kernel<T, 128, 64><<<grid, block, 0, s>>>(p);
-    else if (p.dk == 64 && p.dv == 128) gdn2_decode_kernel<T, 64, 128><<<grid, block, 0, s>>>(p);
-    else if (p.dk == 64 && p.dv == 64) gdn2_decode_kernel<T, 64, 64><<<grid, block, 0, s>>>(p);
+    if (p.dk == 128 && p.dv == 128) gdn2_decode_kernel<T, 128, 128, kRaw><<<grid, block, 0, s>>>(p);
+    else if (p.dk == 128 && p.dv == 64) gdn2_decode_kernel<T, 128, 64, kRaw><<<grid, block, 0, s>>>(p);
+    else if (p.dk == 64 && p.dv == 128) gdn2_decode_kernel<T, 64, 128, kRaw><<<grid, block, 0, s>>>(p);
+    else if (p.dk == 64 && p.dv == 64) gdn2_decode_kernel<T, 64, 64, kRaw><<<grid, block, 0, s>>>(p);
     else return cudaErrorInvalidValue;
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_t(const DecodeParams &p, cudaStream_t s) {
+    return p.qk_raw ? launch_tr<T, true>(p, s) : launch_tr<T, false>(p, s);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t stream) {

@@ -91,20 +91,28 @@ __global__ void __launch_bounds__(256) gdn2_fwd_simt_kernel(FwdParams p) {
         // (a) load the chunk; identity padding past the end of the sequence
         for (int e = tid; e < C * dk; e += NT) {
             const int t = e / dk, i = e % dk;
-            float kv = 0.f, bv = 0.f, qv = 0.f, lv = 0.f;
+            float kv = 0.f, bv = 0.f, qv = 0.f, lv = 0.f, gate = 0.f;
             if (t < n) {
                 const size_t gt = ((size_t)bb * T_ + t0 + t) * H + h;   // token and head
                 const size_t gi = gt * dk + i;
                 kv = ldf(k, gi);
                 bv = beta ? ldf(beta, gt) : ldf(b, gi);
                 const float gs = p.gs ? p.gs[(size_t)h * dk + i] : 1.f;
-                qv = ldf(q, gi) * gs * two_sigmoid(z ? ldf(z, gi) : 0.f);
+                gate = gs * two_sigmoid(z ? ldf(z, gi) : 0.f);
+                qv = ldf(q, gi);
+                if (p.qk_raw) {
+                    kv = silu(kv);
+                    qv = silu(qv);
+                } else {
+                    qv *= gate;
+                }
                 lv = p.decay_tok ? p.la[gt] : p.la[gi];
             }
             sk[t * dkp + i] = kv;
-            skh[t * dkp + i] = bv * kv;
+            skh[t * dkp + i] = p.qk_raw ? bv : bv * kv;   // raw: finished after the norms below
             sqt[t * dkp + i] = qv;
             slam[t * dkp + i] = lv;
+            if (p.qk_raw) stmp[t * dkp + i] = gate;        // stmp is free until (b)
         }
         for (int e = tid; e < C * dv; e += NT) {
             const int t = e / dv, j = e % dv;
@@ -115,6 +123,26 @@ __global__ void __launch_bounds__(256) gdn2_fwd_simt_kernel(FwdParams p) {
                 x = (beta ? ldf(beta, gt) : ldf(w, gi)) * ldf(v, gi);
             }
             svh[t * dv + j] = x;
+        }
+        if (p.qk_raw) {
+            // per-token l2 norms of SiLU(k) and SiLU(q) over the head's d_k channels;
+            // the normalised values are held in the token dtype, then gated
+            __syncthreads();
+            float *sinv = sM;                                 // [2][C]; sM is written only in (c)
+            for (int r = tid; r < 2 * C; r += NT) {
+                const float *row = r < C ? sk + r * dkp : sqt + (r - C) * dkp;
+                float ss = 0.f;
+                for (int i = 0; i < dk; ++i) ss = fmaf(row[i], row[i], ss);
+                sinv[r] = rsqrtf(fmaxf(ss, 1e-24f));
+            }
+            __syncthreads();
+            for (int e = tid; e < C * dk; e += NT) {
+                const int t = e / dk, i = e % dk;
+                const float kn = as_dtype(sk[t * dkp + i] * sinv[t], k);
+                sk[t * dkp + i] = kn;
+                skh[t * dkp + i] *= kn;
+                sqt[t * dkp + i] = as_dtype(sqt[t * dkp + i] * sinv[C + t], q) * stmp[t * dkp + i];
+            }
         }
         __syncthreads();
         // (b) cumulative log-decay and gamma_t = e^{Lambda_t} (<= 1)

@@ -154,6 +154,7 @@ struct TcParams {
     const int *wflags;       // per-window flag: 0 = tiles valid, 1 = process here
     const __nv_bfloat16 *beta;   // one gate per token and head standing for both b and w, or null
     int decay_tok;               // 1: la holds one log-decay per token and head
+    int qk_raw;                  // 1: q and k need SiLU and l2 normalisation
     int NW;                  // windows of 64 tokens per head
 };
 
@@ -165,6 +166,24 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4 &u, float *f) {
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
+}
+
+// Key/query preprocessing on one token row held by a whole warp (four channels
+// a lane, 128 in all): SiLU, division by the row's l2 norm (floored at 1e-12),
+// and rounding to bf16 as a separate normalisation would store the result.
+// Every lane of the warp must call it (full-warp shuffles).
+__device__ __forceinline__ void silu_l2n_row4(float (&f)[4]) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[i] *= 0.5f * two_sigmoid_fast(f[i]);
+        ss = fmaf(f[i], f[i], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(fmaxf(ss, 1e-24f));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = __bfloat162float(__float2bfloat16_rn(f[i] * inv));
 }
 
 // A gate given once per token and head, repeated over four channels as a bf16 quad.
@@ -246,6 +265,9 @@ __device__ __forceinline__ void merge_level(float *lw, float *yb, int tid) {
 // state recurrence moves on to the next chunk.  [R; O] alternates between two
 // TMEM slots; warps 8-9 have no role.
 // ---------------------------------------------------------------------------
+// kRaw: q and k arrive before their SiLU and l2 normalisation (read only by the
+// shorter-chunk path; window records hold the preprocessed operands).
+template <bool kRaw>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gdn2_fwd_tc_kernel(TcParams p) {
     using L = ChainSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -529,6 +551,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                                     f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
                                     f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
                                     f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
+                                }
+                                if (kRaw) {                 // the q/k preprocessing, one token a call
+                                    silu_l2n_row4(kk);
+                                    silu_l2n_row4(qq);
                                 }
                             }
                             float kp[4], kc[4], khc[4], qp[4];
@@ -1020,10 +1046,11 @@ constexpr uint32_t kItmW = 0;      // W' (M=64) reuses the columns of P after it
 constexpr uint32_t kItmN = 128;    // N  (M=64)
 }  // namespace
 
-// Gate forms, fixed at compile time: kNoZ reads no z (2 sigmoid(z) = 1), kBeta
+// Input forms, fixed at compile time: kNoZ reads no z (2 sigmoid(z) = 1), kBeta
 // reads one beta per token and head for both b and w, kTok one log-decay per
-// token and head.  All false is the per-channel GDN-2 form.
-template <bool kNoZ, bool kBeta, bool kTok>
+// token and head, kRaw applies SiLU and l2 normalisation to q and k.  All false
+// is the per-channel GDN-2 form on preprocessed q and k.
+template <bool kNoZ, bool kBeta, bool kTok, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
     using L = IntraSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1180,6 +1207,10 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                         f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
                         f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
                         f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
+                    }
+                    if (kRaw) {                         // the q/k preprocessing, one token a call
+                        silu_l2n_row4(kk);
+                        silu_l2n_row4(qq);
                     }
                 }
                 float kp[4], kc[4], khc[4], qp[4];
@@ -1428,7 +1459,7 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.b = (const __nv_bfloat16 *)fp.b; p.v = (const __nv_bfloat16 *)fp.v; p.w = (const __nv_bfloat16 *)fp.w;
     p.g = (const __nv_bfloat16 *)fp.g;
     p.la = fp.la; p.gs = fp.gs; p.S_in = fp.S_in; p.S_out = fp.S_out;
-    p.beta = (const __nv_bfloat16 *)fp.beta; p.decay_tok = fp.decay_tok;
+    p.beta = (const __nv_bfloat16 *)fp.beta; p.decay_tok = fp.decay_tok; p.qk_raw = fp.qk_raw;
     p.y = (__nv_bfloat16 *)fp.y; p.o_raw = fp.o_raw; p.eps = fp.eps; p.status = fp.status;
     p.NW = (fp.T + kC - 1) / kC;
     const size_t nwin = (size_t)fp.B * fp.H * p.NW;
@@ -1439,22 +1470,26 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
 
     const size_t ismem = (size_t)IntraSmem::TOTAL + 1024;
     using IntraFn = void (*)(TcParams, uint8_t *, int *);
-    static constexpr IntraFn kIntra[8] = {
-        gdn2_chunk_intra_tc_kernel<false, false, false>, gdn2_chunk_intra_tc_kernel<false, false, true>,
-        gdn2_chunk_intra_tc_kernel<false, true, false>,  gdn2_chunk_intra_tc_kernel<false, true, true>,
-        gdn2_chunk_intra_tc_kernel<true, false, false>,  gdn2_chunk_intra_tc_kernel<true, false, true>,
-        gdn2_chunk_intra_tc_kernel<true, true, false>,   gdn2_chunk_intra_tc_kernel<true, true, true>};
-    const IntraFn intra = kIntra[(p.z == nullptr) * 4 + (p.beta != nullptr) * 2 + (p.decay_tok != 0)];
+#define GDN2_INTRA_FORMS(R)                                                                                    \
+    gdn2_chunk_intra_tc_kernel<false, false, false, R>, gdn2_chunk_intra_tc_kernel<false, false, true, R>,    \
+        gdn2_chunk_intra_tc_kernel<false, true, false, R>, gdn2_chunk_intra_tc_kernel<false, true, true, R>,  \
+        gdn2_chunk_intra_tc_kernel<true, false, false, R>, gdn2_chunk_intra_tc_kernel<true, false, true, R>,  \
+        gdn2_chunk_intra_tc_kernel<true, true, false, R>, gdn2_chunk_intra_tc_kernel<true, true, true, R>
+    static constexpr IntraFn kIntra[16] = {GDN2_INTRA_FORMS(false), GDN2_INTRA_FORMS(true)};
+#undef GDN2_INTRA_FORMS
+    const IntraFn intra = kIntra[(p.qk_raw != 0) * 8 + (p.z == nullptr) * 4 + (p.beta != nullptr) * 2 +
+                                 (p.decay_tok != 0)];
     cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ismem);
     if (e != cudaSuccess) return e;
     intra<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)ChainSmem::TOTAL + 1024;
-    e = cudaFuncSetAttribute(gdn2_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto chain = fp.qk_raw ? gdn2_fwd_tc_kernel<true> : gdn2_fwd_tc_kernel<false>;
+    e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // clusters of two CTAs (value-column halves of one head), set by the kernel's attribute
-    gdn2_fwd_tc_kernel<<<2 * fp.B * fp.H, kChainThreads, smem, stream>>>(p);
+    chain<<<2 * fp.B * fp.H, kChainThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

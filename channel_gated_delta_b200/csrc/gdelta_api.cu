@@ -38,7 +38,8 @@ static gdelta_status check_fwd(const gdelta_fwd_args *a, bool need_tensors = tru
     const int C = a->chunk == 0 ? 64 : a->chunk;
     if (C != 16 && C != 32 && C != 64) return GDELTA_ERR_UNSUPPORTED;
     if (a->path < GDELTA_PATH_AUTO || a->path > GDELTA_PATH_TC) return GDELTA_ERR_INVALID_ARG;
-    if (a->reserved2 != 0 || (a->decay_per_token != 0 && a->decay_per_token != 1)) return GDELTA_ERR_INVALID_ARG;
+    if ((a->qk_raw != 0 && a->qk_raw != 1) || (a->decay_per_token != 0 && a->decay_per_token != 1))
+        return GDELTA_ERR_INVALID_ARG;
     if (a->beta && (a->b || a->w)) return GDELTA_ERR_INVALID_ARG;     // one gate form, not both
     if (need_tensors && a->T > 0) {
         if (!a->q || !a->k || !a->v || !a->g || !a->log_alpha || !a->y) return GDELTA_ERR_INVALID_ARG;
@@ -143,7 +144,7 @@ gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     p.q = a->q; p.k = a->k; p.z = a->z; p.b = a->b; p.v = a->v; p.w = a->w; p.g = a->g;
     p.la = a->log_alpha; p.gs = a->gamma_stat; p.S_in = a->S_in; p.S_out = a->S_out;
     p.y = a->y; p.o_raw = a->o_raw; p.eps = a->eps;
-    p.beta = a->beta; p.decay_tok = a->decay_per_token;
+    p.beta = a->beta; p.decay_tok = a->decay_per_token; p.qk_raw = a->qk_raw;
     p.status = status_ptr();
     if (path == GDELTA_PATH_TC) {
         p.C = 64;
@@ -158,7 +159,8 @@ gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
 
 gdelta_status gdelta_decode_step(const gdelta_decode_args *a, void *stream) {
     if (!a) return GDELTA_ERR_INVALID_ARG;
-    if (a->B < 1 || a->H < 1 || a->reserved != 0 || a->reserved2 != 0) return GDELTA_ERR_INVALID_ARG;
+    if (a->B < 1 || a->H < 1 || a->reserved != 0 || (a->qk_raw != 0 && a->qk_raw != 1))
+        return GDELTA_ERR_INVALID_ARG;
     if (a->decay_per_token != 0 && a->decay_per_token != 1) return GDELTA_ERR_INVALID_ARG;
     if (a->beta ? (a->b || a->w) : (!a->b || !a->w)) return GDELTA_ERR_INVALID_ARG;
     if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return GDELTA_ERR_INVALID_ARG;
@@ -174,7 +176,7 @@ gdelta_status gdelta_decode_step(const gdelta_decode_args *a, void *stream) {
     p.q = a->q; p.k = a->k; p.z = a->z; p.b = a->b; p.v = a->v; p.w = a->w; p.g = a->g;
     p.la = a->log_alpha; p.gs = a->gamma_stat; p.S = a->S; p.y = a->y; p.o_raw = a->o_raw;
     p.eps = a->eps;
-    p.beta = a->beta; p.decay_tok = a->decay_per_token;
+    p.beta = a->beta; p.decay_tok = a->decay_per_token; p.qk_raw = a->qk_raw;
     return launch_decode(p, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
                                                                            : GDELTA_ERR_CUDA;
 }

@@ -53,7 +53,7 @@ def compose_affine(A, S, D):
 
 def gdelta_fwd_seqshard(q, k, v, b, w, z, g, log_alpha, *, group=None, S_in=None, gamma_stat=None,
                         y=None, chunk: int = 64, eps: float = 1e-6, path: str = "auto", beta=None,
-                        decay_per_token: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                        decay_per_token: bool = False, qk_raw: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Forward over this rank's segment of one sequence split in rank order.
 
     Tensors are this rank's segment ([B, T_r, H, d]); S_in is the state before
@@ -67,13 +67,13 @@ def gdelta_fwd_seqshard(q, k, v, b, w, z, g, log_alpha, *, group=None, S_in=None
     if world == 1:                                    # one segment: the plain forward
         return gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, gamma_stat=gamma_stat, S_in=S_in, y=y,
                                   chunk=chunk, eps=eps, path=path, stream=stream, beta=beta,
-                                  decay_per_token=decay_per_token)
+                                  decay_per_token=decay_per_token, qk_raw=qk_raw)
     A, D = gdelta_segment_map(q, k, v, b, w, z, g, log_alpha, beta=beta, decay_per_token=decay_per_token,
-                              chunk=chunk, path=path, stream=stream)
+                              qk_raw=qk_raw, chunk=chunk, path=path, stream=stream)
     As, Ds = gather_maps(A, D, group)
     S0 = compose_range(As, Ds, 0, rank, S_in, compose_affine)
     y, S_end = gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, gamma_stat=gamma_stat, S_in=S0, y=y,
                                   chunk=chunk, eps=eps, path=path, stream=stream, beta=beta,
-                                  decay_per_token=decay_per_token)
+                                  decay_per_token=decay_per_token, qk_raw=qk_raw)
     S_final = compose_range(As, Ds, rank + 1, world, S_end, compose_affine)
     return y, S_final

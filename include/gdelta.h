@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GDELTA_ABI_VERSION 2
+#define GDELTA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define GDELTA_API __attribute__((visibility("default")))
@@ -95,6 +95,13 @@ typedef enum gdelta_fwd_path {
  *                to KDA, a scalar decay further to Gated DeltaNet; "Kimi3 =
  *                GPT2 x 22580" §5, §6).  The kernels then read one value per
  *                token and head instead of two d-long rows.
+ *   qk_raw     : 1 = q and k are given before their preprocessing; the kernels
+ *                apply it as they load them: SiLU, then l2 normalisation over
+ *                the head's d_k channels, x / max(||x||, 1e-12) (Muir review
+ *                §2.1: keys and queries pass through SiLU and are l2-normalised
+ *                per head; values are not).  The normalised q and k are held
+ *                in the token dtype, as a separate normalisation would store
+ *                them.  0 = q and k are used as given.
  *   gamma_stat : [H, d_k]        fp32         static readout profile; NULL = ones
  *   S_in       : [B, H, d_k, d_v] fp32        state before token 0; NULL = zeros
  *   S_out      : [B, H, d_k, d_v] fp32        state after token T-1; NULL = not
@@ -131,7 +138,7 @@ typedef struct gdelta_fwd_args {
     size_t workspace_bytes;
     const void *beta;           /* see above; NULL = per-channel b and w */
     int32_t decay_per_token;    /* 1: log_alpha is [B, T, H] */
-    int32_t reserved2;          /* must be 0 */
+    int32_t qk_raw;             /* 0 or 1, see above */
 } gdelta_fwd_args;
 
 /*
@@ -142,7 +149,8 @@ typedef struct gdelta_fwd_args {
  *   q, k, z, b : [B, H, d_k] dtype;  v, w, g : [B, H, d_v] dtype
  *   log_alpha  : [B, H, d_k] fp32 ([B, H] when decay_per_token is 1)
  *   gamma_stat : [H, d_k] fp32 or NULL
- *   z may be NULL; beta ([B, H] dtype) replaces b and w as in gdelta_fwd_args
+ *   z may be NULL; beta ([B, H] dtype) replaces b and w, and qk_raw applies
+ *   the q/k preprocessing, as in gdelta_fwd_args
  *   S          : [B, H, d_k, d_v] fp32, read as S_{t-1}, overwritten with S_t
  *   y          : [B, H, d_v] dtype;  o_raw : [B, H, d_v] fp32 or NULL
  */
@@ -160,7 +168,7 @@ typedef struct gdelta_decode_args {
     float eps;
     const void *beta;           /* NULL = per-channel b and w */
     int32_t decay_per_token;    /* 1: log_alpha is [B, H] */
-    int32_t reserved2;          /* must be 0 */
+    int32_t qk_raw;             /* 0 or 1: as in gdelta_fwd_args */
 } gdelta_decode_args;
 
 /* ABI version of the loaded library (GDELTA_ABI_VERSION it was built with). */

@@ -89,17 +89,38 @@ def all_heads(B: int, H: int) -> List[Tuple[int, int]]:
     return [(b_, h_) for b_ in range(B) for h_ in range(H)]
 
 
+def preprocess_qk(x) -> np.ndarray:
+    """Key and query preprocessing (Muir review §2.1: SiLU, then l2
+    normalisation per head; values are left alone): x sigmoid(x), divided by
+    its l2 norm over the last axis (the head's channels), the norm floored at
+    1e-12 so that a zero row stays zero.  [..., d] in, float64 out."""
+    x = _f64(x)
+    s = x / (1.0 + np.exp(-x))
+    n = np.sqrt(np.sum(s * s, axis=-1, keepdims=True))
+    return s / np.maximum(n, 1e-12)
+
+
+def _with_raw_qk(inputs: Dict) -> Dict:
+    out = dict(inputs)
+    out["q"] = preprocess_qk(inputs["q"])
+    out["k"] = preprocess_qk(inputs["k"])
+    return out
+
+
 def forward(inputs: Dict, heads: Optional[Iterable[Tuple[int, int]]] = None,
-            S0=None, eps: float = 1e-6, n_threads: int = 0) -> Dict[str, np.ndarray]:
+            S0=None, eps: float = 1e-6, n_threads: int = 0, qk_raw: bool = False) -> Dict[str, np.ndarray]:
     """Token-by-token float64 recurrence over the listed heads.
 
     inputs: q,k,v,b,w,z,g,log_alpha as [B,T,H,d] (torch or numpy, any float
     dtype) and optionally gamma_stat [H,dk] (absent or None = ones).
     heads:  list of (b, h); None = all heads in (b, h) order.
     S0:     None (zeros) or [n_heads, dk, dv].
+    qk_raw: q and k are given before ``preprocess_qk``, which is applied first.
     Returns float64 arrays y, o_raw [n_heads, T, dv], S [n_heads, dk, dv] and
     the thread count used under "threads".
     """
+    if qk_raw:
+        inputs = _with_raw_qk(inputs)
     B, T, H, dk = tuple(inputs["q"].shape)
     dv = int(inputs["v"].shape[-1])
     heads = all_heads(B, H) if heads is None else list(heads)
@@ -137,7 +158,7 @@ def forward_full(inputs: Dict, S0=None, eps: float = 1e-6, n_threads: int = 0) -
 
 def decode_steps(step_inputs: Sequence[Dict], S0, gamma_stat=None,
                  heads: Optional[Sequence[Tuple[int, int]]] = None, eps: float = 1e-6,
-                 n_threads: int = 0) -> Dict[str, np.ndarray]:
+                 n_threads: int = 0, qk_raw: bool = False) -> Dict[str, np.ndarray]:
     """Consecutive single-token updates.
 
     step_inputs: one dict per step with [B,H,d] tensors; S0: [n_heads,dk,dv]
@@ -150,7 +171,7 @@ def decode_steps(step_inputs: Sequence[Dict], S0, gamma_stat=None,
     for inp in step_inputs:
         tok = {key: inp[key][:, None] for key in TOKEN_KEYS}
         tok["gamma_stat"] = gamma_stat
-        r = forward(tok, heads, S, eps, n_threads)
+        r = forward(tok, heads, S, eps, n_threads, qk_raw=qk_raw)
         S = r["S"]
         ys.append(r["y"][:, 0])
         os_.append(r["o_raw"][:, 0])

@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.gdelta_abi_version() == 2
+    assert lib.gdelta_abi_version() == 3
     for code in range(8):
         s = lib.gdelta_status_string(code)
         assert s and s != b"unknown status"
@@ -90,10 +90,10 @@ def test_reduced_gate_forms_are_validated_on_the_host(lib):
     assert f(ctypes.byref(_args(b=None)), None) == 1
     assert f(ctypes.byref(_args(w=None)), None) == 1
     assert f(ctypes.byref(_args(decay_per_token=2)), None) == 1
-    assert f(ctypes.byref(_args(reserved2=1)), None) == 1
+    assert f(ctypes.byref(_args(qk_raw=2)), None) == 1
     assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(beta=beta))) == -1
     # accepted forms: no z; beta alone; beta with a per-token decay
-    for kw in ({"z": None}, {"b": None, "w": None, "beta": beta},
+    for kw in ({"z": None}, {"qk_raw": 1}, {"b": None, "w": None, "beta": beta},
                {"b": None, "w": None, "beta": beta, "decay_per_token": 1, "z": None}):
         assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(**kw))) in (1, 2), kw
         assert lib.gdelta_fwd_workspace_bytes(ctypes.byref(_args(**kw))) >= 0
@@ -104,9 +104,9 @@ def test_reduced_gate_forms_are_validated_on_the_host(lib):
     d.eps = 1e-6
     d.beta = beta
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # beta beside b and w
-    d.beta, d.reserved2 = None, 1
+    d.beta, d.qk_raw = None, 2
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
-    d.reserved2, d.decay_per_token = 0, 5
+    d.qk_raw, d.decay_per_token = 0, 5
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1
     d.decay_per_token, d.b = 0, None
     assert lib.gdelta_decode_step(ctypes.byref(d), None) == 1       # b missing, no beta

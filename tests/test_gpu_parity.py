@@ -488,3 +488,88 @@ def test_seqshard_segments_compose_to_the_whole_sequence(dtype, path, dk, dv):
     assert err_stored(sel_heads(torch.cat(ys, 1).cpu(), heads), ref["y"], dtype) <= tol
     for S_fin in finals:                              # every rank ends with the sequence's final state
         assert err(S_fin.cpu().reshape(H, dk, dv), ref["S"]) <= tol
+
+
+# --------------------------------------------------------------------------
+# Raw q and k (qk_raw): the kernels apply SiLU and the per-head l2
+# normalisation as they load them; the oracle applies its own preprocessing.
+# --------------------------------------------------------------------------
+
+def _raw_qk(inp, seed):
+    """Pre-activation q and k: seeded normal draws in the token dtype."""
+    gen = torch.Generator().manual_seed(seed)
+    out = dict(inp)
+    for key in ("q", "k"):
+        out[key] = (torch.randn(inp[key].shape, generator=gen) * 1.5).to(inp[key].dtype)
+    return out
+
+
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_raw_qk_prologue_bf16(path):
+    shape = synth.GdnShape(B=2, T=64 * 3 + 29, H=2, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=101)
+    inp = _raw_qk(synth.generate(shape), 5)
+    y, S, o = gpu_fwd(inp, path=path, qk_raw=True)
+    heads = oracle.all_heads(2, 2)
+    _check(y, S, o, oracle.forward(inp, heads=heads, qk_raw=True), heads, TOL_BF16)
+
+
+def test_raw_qk_prologue_f32():
+    shape = synth.GdnShape(B=1, T=101, H=2, dk=64, dv=128, dtype="f32", seed=102)
+    inp = _raw_qk(synth.generate(shape), 6)
+    y, S, o = gpu_fwd(inp, path="simt", chunk=32, qk_raw=True)
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, oracle.forward(inp, heads=heads, qk_raw=True), heads, TOL_F32)
+
+
+def test_tc_raw_qk_with_shortened_windows_and_reduced_gates():
+    """The chain's own shorter chunks preprocess q and k too; with the Gated
+    DeltaNet gate form on top (every intra switch on)."""
+    shape = synth.GdnShape(B=1, T=64 * 5 + 3, H=2, dk=128, dv=128, dtype="bf16", seed=103)
+    ker, ref_in, tok = _reduce(_raw_qk(synth.generate(shape), 7), "gdn")
+    for side in (ker, ref_in):
+        la = side["log_alpha"].clone()
+        la[:, 64:128] *= 40.0
+        side["log_alpha"] = la
+    y, S, o = _fwd_reduced(ker, tok, path="tc", qk_raw=True)
+    heads = oracle.all_heads(1, 2)
+    _check(y, S, o, oracle.forward(ref_in, heads=heads, qk_raw=True), heads, TOL_BF16)
+
+
+def test_decode_raw_qk():
+    import channel_gated_delta_b200 as gd
+    B, H, dk, dv = 3, 2, 128, 128
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(8)) * 0.3
+    S = S0.cuda()
+    heads = oracle.all_heads(B, H)
+    Sref = S0.reshape(B * H, dk, dv).double().numpy()
+    for s in range(4):
+        inp = _raw_qk(synth.decode_step_inputs(s, seed=104, B=B, H=H, dk=dk, dv=dv), 20 + s)
+        d = to_dev(inp)
+        y = gd.gdelta_decode_step(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], S,
+                                  qk_raw=True)
+        ref = oracle.decode_steps([inp], Sref, heads=heads, qk_raw=True)
+        Sref = ref["S"]
+        assert err_stored(y.cpu().reshape(B * H, dv), ref["y"][0], "bf16") <= TOL_BF16
+    assert err(S.cpu().reshape(B * H, dk, dv), Sref) <= TOL_BF16
+
+
+def test_segment_map_with_raw_qk_composes():
+    """The segment maps read raw q and k the same way as the forward."""
+    import channel_gated_delta_b200 as gd
+    from channel_gated_delta_b200.seqshard import compose_affine, compose_range
+    bounds, H = [0, 131, 300], 2
+    inp = _raw_qk(synth.generate(synth.GdnShape(B=1, T=300, H=H, dk=128, dv=128, dtype="bf16", seed=105)), 9)
+    d = to_dev(inp)
+    segs = [{k: (v[:, bounds[r]:bounds[r + 1]] if v.dim() == 4 else v) for k, v in d.items()} for r in range(2)]
+    maps = [gd.gdelta_segment_map(s["q"], s["k"], s["v"], s["b"], s["w"], s["z"], s["g"], s["log_alpha"],
+                                  qk_raw=True, path="tc") for s in segs]
+    As, Ds = [m[0] for m in maps], [m[1] for m in maps]
+    S0 = compose_range(As, Ds, 0, 1, None, compose_affine)
+    s = segs[1]
+    y, S_end = gd.gdelta_fwd_chunked(s["q"], s["k"], s["v"], s["b"], s["w"], s["z"], s["g"], s["log_alpha"],
+                                     gamma_stat=d["gamma_stat"], S_in=S0, path="tc", qk_raw=True)
+    torch.cuda.synchronize()
+    heads = oracle.all_heads(1, H)
+    ref = oracle.forward(inp, heads=heads, qk_raw=True)
+    assert err_stored(sel_heads(y.cpu(), heads), ref["y"][:, 131:], "bf16") <= TOL_BF16
+    assert err(S_end.cpu().reshape(H, 128, 128), ref["S"]) <= TOL_BF16

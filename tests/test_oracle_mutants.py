@@ -10,6 +10,7 @@ import os
 import subprocess
 import tempfile
 
+import numpy as np
 import pytest
 
 import oracle
@@ -139,3 +140,46 @@ def test_unmodified_source_passes_every_pin():
     for call in PIN_CALLS:
         call()
     assert oracle._lib is real
+
+
+# Mistakes in the q/k preprocessing (a Python step of the oracle), planted by
+# swapping the function for a wrong one; the preprocessing pins must notice.
+def _prep_no_silu(x):
+    x = oracle._f64(x)
+    return x / np.maximum(np.linalg.norm(x, axis=-1, keepdims=True), 1e-12)
+
+
+def _prep_sigmoid(x):
+    x = oracle._f64(x)
+    s = 1.0 / (1.0 + np.exp(-x))
+    return s / np.maximum(np.linalg.norm(s, axis=-1, keepdims=True), 1e-12)
+
+
+def _prep_wrong_axis(x):
+    x = oracle._f64(x)
+    s = x / (1.0 + np.exp(-x))
+    return s / np.maximum(np.linalg.norm(s, axis=0, keepdims=True), 1e-12)
+
+
+def _prep_no_floor(x):
+    x = oracle._f64(x)
+    s = x / (1.0 + np.exp(-x))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return s / np.linalg.norm(s, axis=-1, keepdims=True)
+
+
+PREP_MUTANTS = {"no_silu": _prep_no_silu, "sigmoid_not_silu": _prep_sigmoid,
+                "normalised_over_the_wrong_axis": _prep_wrong_axis, "no_norm_floor": _prep_no_floor}
+
+
+@pytest.mark.parametrize("name", sorted(PREP_MUTANTS))
+def test_preprocessing_pins_catch_mutant(name, monkeypatch):
+    monkeypatch.setattr(oracle, "preprocess_qk", PREP_MUTANTS[name])
+    failed = 0
+    for pin in (pins.test_preprocess_qk_is_unit_norm_along_the_head_channels,
+                pins.test_preprocess_qk_direction_is_silu, pins.test_preprocess_qk_special_rows):
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed >= 1, name

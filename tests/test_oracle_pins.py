@@ -410,3 +410,61 @@ def test_head_selection_and_full_layout():
     sel = oracle.forward(d, heads=[(1, 2), (0, 1)])
     assert np.array_equal(sel["y"][0], full["y"][1, :, 2])
     assert np.array_equal(sel["S"][1], full["S"][0, 1])
+
+
+# --------------------------------------------------------------------------
+# Key/query preprocessing (Muir review §2.1: SiLU, then l2 normalisation per
+# head; values untouched), pinned by what fixes it rather than by retyping it
+# --------------------------------------------------------------------------
+
+def test_preprocess_qk_is_unit_norm_along_the_head_channels():
+    rng = np.random.Generator(np.random.PCG64(5))
+    x = rng.standard_normal((3, 7, 2, 64)) * 3.0
+    y = oracle.preprocess_qk(x)
+    assert np.allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-12)
+    # normalised over the last axis only: scaling one token row leaves the others alone
+    x2 = x.copy()
+    x2[1, 3, 0] *= 5.0
+    y2 = oracle.preprocess_qk(x2)
+    mask = np.ones(x.shape[:-1], bool)
+    mask[1, 3, 0] = False
+    assert np.array_equal(y2[mask], y[mask])
+
+
+def test_preprocess_qk_direction_is_silu():
+    """Parallel to x * logistic(x), the logistic taken from scipy."""
+    from scipy.special import expit
+    rng = np.random.Generator(np.random.PCG64(6))
+    x = rng.standard_normal((5, 32)) * 4.0
+    s = x * expit(x)
+    y = oracle.preprocess_qk(x)
+    cos = np.sum(y * s, axis=-1) / np.linalg.norm(s, axis=-1)
+    assert np.allclose(cos, 1.0, atol=1e-12)
+    # SiLU is not odd: a row and its negation do not map to opposite rows
+    assert not np.allclose(oracle.preprocess_qk(-x), -y)
+
+
+def test_preprocess_qk_special_rows():
+    e = np.zeros((3, 8))
+    e[0, 2] = 1.5                     # one positive channel -> that unit vector
+    e[1, 5] = -2.0                    # one negative channel: SiLU < 0 -> minus that unit vector
+    y = oracle.preprocess_qk(e)       # row 2 all zero: stays zero (the norm floor)
+    assert np.allclose(y[0], np.eye(8)[2]) and np.allclose(y[1], -np.eye(8)[5])
+    assert np.array_equal(y[2], np.zeros(8))
+
+
+def test_forward_qk_raw_applies_the_preprocessing_first():
+    """The raw-input forward equals the forward on preprocessed q and k, and a
+    plain forward on the raw tensors differs (the flag is not ignored)."""
+    import synth
+    inp = synth.generate(synth.GdnShape(B=1, T=40, H=2, dk=32, dv=16, dtype="f32", seed=3))
+    rng = np.random.Generator(np.random.PCG64(7))
+    raw = dict(inp)
+    raw["q"] = rng.standard_normal(inp["q"].shape)
+    raw["k"] = rng.standard_normal(inp["k"].shape)
+    pre = dict(raw)
+    pre["q"], pre["k"] = oracle.preprocess_qk(raw["q"]), oracle.preprocess_qk(raw["k"])
+    a = oracle.forward(raw, qk_raw=True)
+    b = oracle.forward(pre)
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["S"], b["S"])
+    assert not np.allclose(oracle.forward(raw)["y"], a["y"])
