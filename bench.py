@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--stream-tokens", type=int, default=0,
                     help="also serve one long stream (B1 H16) of this many tokens: forward calls of "
                          "16384 tokens carrying the state, then decode steps (0 = off)")
+    ap.add_argument("--bwd-calls", type=int, default=2,
+                    help="timed gdelta_bwd calls on the workload (0 = skip the backward measurement)")
     ap.add_argument("--no-forms", action="store_true",
                     help="skip the forward timings of the reduced gate forms")
     # profiling aid: a smaller case of the same workload (fewer batch rows) for
@@ -286,6 +288,9 @@ def run_ours(args, rank, local, world):
     # ---- forward alone on the reduced gate forms (same workload shape)
     forms = None if args.no_forms else run_forms(args, gd, d, shape, dev, stream, ws, world)
 
+    # ---- backward pass on the same workload
+    bwd = run_bwd(args, gd, d, shape, dev, stream, world) if args.bwd_calls > 0 else None
+
     # ---- one long stream: consecutive forward calls, then decode (opt-in)
     stream_res = run_stream(args, gd, d, shape, dev, stream, world) if args.stream_tokens > 0 else None
 
@@ -343,6 +348,7 @@ def run_ours(args, rank, local, world):
         "decode": dec,
         "forms": forms,
         "stream": stream_res,
+        "backward": bwd,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -475,6 +481,48 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
             out[name]["torch_preprocess_then_fwd_ms_median"] = max_over_ranks(
                 statistics.median(a.elapsed_time(c) for a, c in ev2), world)
     return out
+
+
+def bwd_bytes(B, T, H, dk, dv, tok_bytes):
+    """Algorithmic HBM bytes of one backward call: the forward's inputs (q, k,
+    z, b, v, w, g, log_alpha) and dL/dy read once, the eight fp32 token
+    gradients written, the states S_in and dL/dS_out read and dL/dS_in written."""
+    per = 4 * dk * tok_bytes + 3 * dv * tok_bytes + 4 * dk + 4 * dv + 4 * (5 * dk + 3 * dv)
+    return B * T * H * per + 3 * B * H * dk * dv * 4 + 2 * H * dk * 4
+
+
+def run_bwd(args, gd, d, shape, dev, stream, world):
+    """gdelta_bwd on the workload (dL/dy random, dL/dS_T zero), CUDA events."""
+    B, T, H, dk, dv = shape.B, shape.T, shape.H, shape.dk, shape.dv
+    gen = torch.Generator(device="cpu").manual_seed(13)
+    dy = torch.randn(B, T, H, dv, generator=gen).to(dev)
+    S0 = torch.zeros(B, H, dk, dv, device=dev)
+
+    def call():
+        # outputs and workspace come from torch's caching allocator (no cudaMalloc after the warm-up)
+        return gd.gdelta_bwd(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], dy,
+                             gamma_stat=d["gamma_stat"], S_in=S0, stream=stream)
+
+    call()                                                # warm-up
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.bwd_calls)]
+    barrier(world)
+    for a, c in evs:
+        a.record(stream)
+        call()
+        c.record(stream)
+    torch.cuda.synchronize(dev)
+    if gd.gdelta_get_last_device_error(stream) != 0:
+        raise RuntimeError("device status word set during the backward")
+    ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
+    nb = bwd_bytes(B, T, H, dk, dv, 2)
+    hbm, _ = peaks()
+    gbs = nb / (ms * 1e-3) / 1e9
+    return {"kernel": "gdn2_bwd_kernel (+ gdn2_bwd_dgamma_kernel)", "ms_per_call": ms,
+            "tokens_per_s": B * T * world / (ms * 1e-3), "algorithmic_bytes": nb,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
+            "timed_calls": args.bwd_calls,
+            "note": "one CTA per head walks its tokens in order: latency-bound, 64 of 148 SMs busy"}
 
 
 def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):

@@ -34,6 +34,7 @@ __all__ = [
     "gdelta_segment_map",
     "gdelta_fwd_chunked",
     "gdelta_decode_step",
+    "gdelta_bwd",
     "gdelta_get_last_device_error",
 ]
 
@@ -277,6 +278,46 @@ def gdelta_decode_step(q, k, v, b, w, z, g, log_alpha, S, *, gamma_stat=None, y=
     a.eps = float(eps)
     _check(_lib().gdelta_decode_step(ctypes.byref(a), _stream(stream)), "gdelta_decode_step")
     return y
+
+
+def gdelta_bwd(q, k, v, b, w, z, g, log_alpha, grad_y, *, gamma_stat=None, S_in=None, grad_S_out=None,
+               eps: float = 1e-6, workspace=None, stream=None) -> dict:
+    """Gradients of a loss L given dL/dy (grad_y [B,T,H,dv] fp32) and
+    optionally dL/dS_T (grad_S_out [B,H,dk,dv] fp32), for the forward
+    gdelta_fwd_chunked(q, k, v, b, w, z, g, log_alpha, gamma_stat=..., S_in=...)
+    computes (d_k = d_v = 128).  Returns fp32 tensors under the keys q, k, v,
+    b, w, z, g, log_alpha, gamma_stat ([H,dk]) and S_in ([B,H,dk,dv])."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    dev = q.device
+    ks, vs = (B, T, H, dk), (B, T, H, dv)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {n: torch.empty(ks, **f32) for n in ("q", "k", "z", "b", "log_alpha")}
+    out.update({n: torch.empty(vs, **f32) for n in ("v", "w", "g")})
+    out["gamma_stat"] = torch.empty((H, dk), **f32)
+    out["S_in"] = torch.empty((B, H, dk, dv), **f32)
+    a = _native.BwdArgs()
+    a.B, a.T, a.H, a.dk, a.dv = int(B), int(T), int(H), int(dk), int(dv)
+    a.dtype = _dtype_code(q)
+    for n, t, shp in (("q", q, ks), ("k", k, ks), ("z", z, ks), ("b", b, ks), ("v", v, vs), ("w", w, vs),
+                      ("g", g, vs)):
+        setattr(a, n, _dev_ptr(t, n, dt, shp))
+    a.log_alpha = _dev_ptr(log_alpha, "log_alpha", torch.float32, ks)
+    a.gamma_stat = _dev_ptr(gamma_stat, "gamma_stat", torch.float32, (H, dk), required=False)
+    a.S_in = _dev_ptr(S_in, "S_in", torch.float32, (B, H, dk, dv), required=False)
+    a.grad_y = _dev_ptr(grad_y, "grad_y", torch.float32, vs)
+    a.grad_S_out = _dev_ptr(grad_S_out, "grad_S_out", torch.float32, (B, H, dk, dv), required=False)
+    a.eps = float(eps)
+    for n in ("q", "k", "z", "b", "log_alpha", "v", "w", "g", "gamma_stat", "S_in"):
+        setattr(a, "grad_" + n, out[n].data_ptr())
+    need = int(_lib().gdelta_bwd_workspace_bytes(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    a.workspace = _dev_ptr(workspace, "workspace")
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib().gdelta_bwd(ctypes.byref(a), _stream(stream)), "gdelta_bwd")
+    return out
 
 
 def gdelta_get_last_device_error(stream=None) -> int:

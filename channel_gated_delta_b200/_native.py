@@ -37,6 +37,8 @@ EXPORTED = (
     "gdelta_fwd_chunked",
     "gdelta_fwd_chunked_noalloc",
     "gdelta_decode_step",
+    "gdelta_bwd_workspace_bytes",
+    "gdelta_bwd",
     "gdelta_get_last_device_error",
 )
 
@@ -70,6 +72,20 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class BwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("q", _vp), ("k", _vp), ("z", _vp), ("b", _vp), ("v", _vp), ("w", _vp), ("g", _vp),
+        ("log_alpha", _fp), ("gamma_stat", _fp), ("S_in", _fp),
+        ("grad_y", _fp), ("grad_S_out", _fp), ("eps", ctypes.c_float),
+        ("grad_q", _fp), ("grad_k", _fp), ("grad_z", _fp), ("grad_b", _fp), ("grad_log_alpha", _fp),
+        ("grad_v", _fp), ("grad_w", _fp), ("grad_g", _fp),
+        ("grad_gamma_stat", _fp), ("grad_S_in", _fp),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _lib = None
 
 
@@ -100,6 +116,10 @@ def load(path: str = LIB_PATH):
     lib.gdelta_fwd_chunked.argtypes = [ctypes.POINTER(FwdArgs), _vp]
     lib.gdelta_fwd_chunked_noalloc.restype = ctypes.c_int
     lib.gdelta_fwd_chunked_noalloc.argtypes = [ctypes.POINTER(FwdArgs), _vp]
+    lib.gdelta_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdelta_bwd_workspace_bytes.argtypes = [ctypes.POINTER(BwdArgs)]
+    lib.gdelta_bwd.restype = ctypes.c_int
+    lib.gdelta_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp]
     lib.gdelta_decode_step.restype = ctypes.c_int
     lib.gdelta_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
     lib.gdelta_get_last_device_error.restype = ctypes.c_int

@@ -72,12 +72,26 @@ struct DecodeParams {
     int qk_raw;
 };
 
+// Backward pass (d_k = d_v = 128): forward inputs, the incoming gradients,
+// the gradient outputs (fp32) and the workspace partition.
+struct BwdParams {
+    int B, T, H;
+    const void *q, *k, *z, *b, *v, *w, *g;
+    const float *la, *gs, *S_in;
+    const float *dy, *dS_out;
+    float eps;
+    float *grad_q, *grad_k, *grad_v, *grad_b, *grad_w, *grad_z, *grad_g, *grad_la, *grad_gs, *grad_S_in;
+    float *ws_ckpt, *ws_chunk, *ws_dgam;
+};
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
 size_t fwd_simt_smem_bytes(int dk, int dv, int C);
 int fwd_simt_chunk(int dk, int dv, int requested);
 cudaError_t launch_state_init(float *S, const float *src, size_t n, cudaStream_t stream);
+size_t bwd_workspace_bytes(int B, int H, int T);
+cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t stream);
 cudaError_t launch_state_affine(float *S_out, const float *A, const float *S_in, const float *D, int BH, int dk,
                                 int dv, cudaStream_t stream);
 cudaError_t launch_fwd_tc(const FwdParams &p, void *workspace, cudaStream_t stream);

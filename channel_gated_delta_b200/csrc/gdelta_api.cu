@@ -126,6 +126,49 @@ gdelta_status gdelta_state_affine(float *S_out, const float *A, const float *S_i
                : GDELTA_ERR_CUDA;
 }
 
+static gdelta_status check_bwd(const gdelta_bwd_args *a) {
+    if (!a) return GDELTA_ERR_INVALID_ARG;
+    if (a->B < 1 || a->H < 1 || a->T < 0) return GDELTA_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.f) || !std::isfinite(a->eps)) return GDELTA_ERR_INVALID_ARG;
+    if (a->dtype != GDELTA_F32 && a->dtype != GDELTA_BF16) return GDELTA_ERR_UNSUPPORTED;
+    if (a->dk != 128 || a->dv != 128) return GDELTA_ERR_UNSUPPORTED;
+    if (a->T > 0) {
+        const void *req[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->grad_y,
+                             a->grad_q, a->grad_k, a->grad_z, a->grad_b, a->grad_log_alpha,
+                             a->grad_v, a->grad_w, a->grad_g};
+        for (const void *p : req)
+            if (!p) return GDELTA_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->gamma_stat, a->S_in,
+                          a->grad_y, a->grad_S_out, a->grad_q, a->grad_k, a->grad_z, a->grad_b,
+                          a->grad_log_alpha, a->grad_v, a->grad_w, a->grad_g, a->grad_gamma_stat,
+                          a->grad_S_in, a->workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
+    return GDELTA_OK;
+}
+
+size_t gdelta_bwd_workspace_bytes(const gdelta_bwd_args *a) {
+    if (check_bwd(a) != GDELTA_OK) return 0;
+    return bwd_workspace_bytes(a->B, a->H, a->T);
+}
+
+gdelta_status gdelta_bwd(const gdelta_bwd_args *a, void *stream) {
+    const gdelta_status st = check_bwd(a);
+    if (st != GDELTA_OK) return st;
+    if (!a->workspace || a->workspace_bytes < bwd_workspace_bytes(a->B, a->H, a->T)) return GDELTA_ERR_WORKSPACE;
+    BwdParams p{};
+    p.B = a->B; p.T = a->T; p.H = a->H;
+    p.q = a->q; p.k = a->k; p.z = a->z; p.b = a->b; p.v = a->v; p.w = a->w; p.g = a->g;
+    p.la = a->log_alpha; p.gs = a->gamma_stat; p.S_in = a->S_in;
+    p.dy = a->grad_y; p.dS_out = a->grad_S_out; p.eps = a->eps;
+    p.grad_q = a->grad_q; p.grad_k = a->grad_k; p.grad_v = a->grad_v; p.grad_b = a->grad_b;
+    p.grad_w = a->grad_w; p.grad_z = a->grad_z; p.grad_g = a->grad_g; p.grad_la = a->grad_log_alpha;
+    p.grad_gs = a->grad_gamma_stat; p.grad_S_in = a->grad_S_in;
+    return launch_bwd(p, a->workspace, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
+                                                                                    : GDELTA_ERR_CUDA;
+}
+
 gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     gdelta_status st = check_fwd(a);
     if (st != GDELTA_OK) return st;

@@ -214,6 +214,48 @@ GDELTA_API gdelta_status gdelta_state_init(float *S, int32_t B, int32_t H, int32
 GDELTA_API gdelta_status gdelta_state_affine(float *S_out, const float *A, const float *S_in, const float *D,
                                              int32_t B, int32_t H, int32_t dk, int32_t dv, void *stream);
 
+/*
+ * Backward pass: gradients of a loss with respect to every input of
+ * gdelta_fwd_chunked, the static readout profile and the initial state, given
+ * the loss's gradient with respect to y (and optionally the final state).  The
+ * per-channel GDN-2 form with preprocessed q and k (Muir review §2.1), d_k =
+ * d_v = 128; the pages describe a chunked custom backward (Muir review §2.4,
+ * keeping the block inverse and solutions and recomputing boundary decays);
+ * this one recomputes states from checkpoints every 32 tokens instead and
+ * runs the exact per-token gradient recurrence on CUDA cores.
+ *
+ *   B, T, H, dk, dv, dtype, q, k, z, b, v, w, g, log_alpha, gamma_stat,
+ *   S_in, eps   : as in gdelta_fwd_args (gamma_stat, S_in may be NULL)
+ *   grad_y      : [B, T, H, d_v] fp32, dL/dy
+ *   grad_S_out  : [B, H, d_k, d_v] fp32 or NULL (zero), dL/dS_T
+ *   grad_q, grad_k, grad_z, grad_b, grad_log_alpha : [B, T, H, d_k] fp32 out
+ *   grad_v, grad_w, grad_g                         : [B, T, H, d_v] fp32 out
+ *   grad_gamma_stat : [H, d_k] fp32 out (summed over batch and tokens) or NULL
+ *   grad_S_in       : [B, H, d_k, d_v] fp32 out or NULL
+ *   workspace       : gdelta_bwd_workspace_bytes(args) bytes of device memory
+ *                     (checkpoints and one chunk of states per head);
+ *                     GDELTA_ERR_WORKSPACE if smaller
+ * Unsupported shapes return GDELTA_ERR_UNSUPPORTED.  Asynchronous on `stream`.
+ */
+typedef struct gdelta_bwd_args {
+    int32_t B, T, H, dk, dv, dtype;
+    const void *q, *k, *z, *b, *v, *w, *g;
+    const float *log_alpha, *gamma_stat, *S_in;
+    const float *grad_y, *grad_S_out;
+    float eps;
+    float *grad_q, *grad_k, *grad_z, *grad_b, *grad_log_alpha;
+    float *grad_v, *grad_w, *grad_g;
+    float *grad_gamma_stat, *grad_S_in;
+    void *workspace;
+    size_t workspace_bytes;
+} gdelta_bwd_args;
+
+/* Workspace gdelta_bwd needs for these arguments (0 if they are invalid). */
+GDELTA_API size_t gdelta_bwd_workspace_bytes(const gdelta_bwd_args *args);
+
+/* Backward pass; see gdelta_bwd_args. */
+GDELTA_API gdelta_status gdelta_bwd(const gdelta_bwd_args *args, void *stream);
+
 /* Chunked forward; see gdelta_fwd_args. */
 GDELTA_API gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *args, void *stream);
 

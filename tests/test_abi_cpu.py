@@ -126,6 +126,38 @@ def test_state_affine_validation(lib):
     assert f(S, A, S_in, S + 16, 1, 1, 128, 128, None) == 1          # D partly over S_out
 
 
+def _bwd_args(**kw):
+    a = _native.BwdArgs()
+    a.B, a.T, a.H, a.dk, a.dv, a.dtype = 1, 64, 1, 128, 128, 1
+    names = ("q", "k", "z", "b", "v", "w", "g", "log_alpha", "grad_y", "grad_q", "grad_k", "grad_z",
+             "grad_b", "grad_log_alpha", "grad_v", "grad_w", "grad_g")
+    for i, n in enumerate(names):
+        setattr(a, n, 0x100000 + 0x1000 * i)
+    a.eps = 1e-6
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def test_backward_validation(lib):
+    f, wsb = lib.gdelta_bwd, lib.gdelta_bwd_workspace_bytes
+    assert f(None, None) == 1
+    assert f(ctypes.byref(_bwd_args(dk=64)), None) == 2                # d_k = d_v = 128 only
+    assert f(ctypes.byref(_bwd_args(dtype=5)), None) == 2
+    assert f(ctypes.byref(_bwd_args(grad_y=None)), None) == 1
+    assert f(ctypes.byref(_bwd_args(grad_k=None)), None) == 1
+    assert f(ctypes.byref(_bwd_args(q=0x100004)), None) == 3
+    assert f(ctypes.byref(_bwd_args(eps=float("inf"))), None) == 1
+    need = wsb(ctypes.byref(_bwd_args()))
+    # checkpoints (2 for 64 tokens, plus one spare) and 33 chunk states of 64 KiB, and 128 floats
+    assert need == (3 + 33) * 128 * 128 * 4 + 128 * 4
+    assert f(ctypes.byref(_bwd_args(workspace=0x900000, workspace_bytes=need - 1)), None) == 6
+    assert wsb(ctypes.byref(_bwd_args(dk=64))) == 0
+    # no tokens: token tensors may be null
+    empty = {n: None for n in ("q", "k", "z", "b", "v", "w", "g", "log_alpha", "grad_y")}
+    assert wsb(ctypes.byref(_bwd_args(T=0, **empty))) > 0
+
+
 def test_path_selection_is_host_logic(lib):
     a = _args()
     assert lib.gdelta_fwd_selected_path(ctypes.byref(a)) in (1, 2)

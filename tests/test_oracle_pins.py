@@ -468,3 +468,60 @@ def test_forward_qk_raw_applies_the_preprocessing_first():
     b = oracle.forward(pre)
     assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["S"], b["S"])
     assert not np.allclose(oracle.forward(raw)["y"], a["y"])
+
+
+# --------------------------------------------------------------------------
+# Gradient oracle (oracle.backward): its forward is the C recurrence's, and
+# its gradients are the central finite differences of that forward.
+# --------------------------------------------------------------------------
+
+def _bwd_case(T, dk, dv, seed, H=2):
+    import synth
+    inp = synth.generate(synth.GdnShape(B=1, T=T, H=H, dk=dk, dv=dv, dtype="f32", u_low=-4, u_high=0, seed=seed))
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    inp = {key: np.asarray(val, dtype=np.float64) for key, val in inp.items()}
+    dy = rng.standard_normal((1, T, H, dv))
+    dS = rng.standard_normal((H, dk, dv))
+    S0 = rng.standard_normal((H, dk, dv)) * 0.5
+    return inp, dy, dS, S0
+
+
+def test_backward_oracle_forward_is_the_c_recurrence():
+    from oracle import backward as ob
+    inp, dy, dS, S0 = _bwd_case(37, 16, 8, 31)
+    r = ob.backward(inp, dy, dS_out=dS, S0=S0)
+    c = oracle.forward(inp, S0=S0)
+    assert np.max(np.abs(r["y"] - c["y"])) <= 1e-12 * np.max(np.abs(c["y"]))
+    assert np.max(np.abs(r["S"] - c["S"])) <= 1e-12 * np.max(np.abs(c["S"]))
+
+
+def test_backward_oracle_matches_central_differences():
+    """Every coordinate of every input, the static profile and the initial
+    state, on a tiny case: (L(x + h) - L(x - h)) / 2h against the gradient."""
+    import torch
+    from oracle import backward as ob
+    T, dk, dv, H = 6, 5, 4, 1
+    inp, dy, dS, S0 = _bwd_case(T, dk, dv, 41, H=H)
+    inp["gamma_stat"] = np.exp(0.3 * np.random.Generator(np.random.PCG64(5)).standard_normal((H, dk)))
+    g = ob.backward(inp, dy, dS_out=dS, S0=S0)
+
+    def loss(x):
+        args = [torch.as_tensor(x[key][0].transpose(1, 0, 2)) for key in ob.TOKEN_KEYS]   # [H, T, d]
+        y, S = ob.forward_torch(*args, torch.as_tensor(x["gamma_stat"]), torch.as_tensor(x["S0"]), 1e-6)
+        return float((y.numpy() * dy[0].transpose(1, 0, 2)).sum() + (S.numpy() * dS).sum())
+
+    base = dict(inp, S0=S0)
+    h = 1e-6
+    for key in list(ob.TOKEN_KEYS) + ["gamma_stat", "S0"]:
+        grad = g["dS_in"] if key == "S0" else g["d" + key]
+        if key in ob.TOKEN_KEYS:
+            grad = grad[:, :, None, :].transpose(2, 1, 0, 3)     # [n, T, d] -> [1, T, H, d]
+        fd = np.zeros_like(base[key])
+        for idx in np.ndindex(*base[key].shape):
+            xp = {kk: vv.copy() for kk, vv in base.items()}
+            xm = {kk: vv.copy() for kk, vv in base.items()}
+            xp[key][idx] += h
+            xm[key][idx] -= h
+            fd[idx] = (loss(xp) - loss(xm)) / (2 * h)
+        scale = max(np.max(np.abs(fd)), 1e-12)
+        assert np.max(np.abs(fd - grad.reshape(fd.shape))) <= 1e-6 * scale, key
