@@ -522,7 +522,7 @@ def run_bwd(args, gd, d, shape, dev, stream, world):
             "tokens_per_s": B * T * world / (ms * 1e-3), "algorithmic_bytes": nb,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
             "timed_calls": args.bwd_calls,
-            "note": "one CTA per head walks its tokens in order: latency-bound, 64 of 148 SMs busy"}
+            "note": f"one CTA per head walks its tokens in order: latency-bound, {B * H} CTAs"}
 
 
 def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):
