@@ -69,3 +69,58 @@ def test_segment_maps_compose_across_ranks(world, T, dk, dv):
     for r in range(world):
         e_y, e_s = out[r]
         assert e_y < 1e-9 and e_s < 1e-9, (r, e_y, e_s)
+
+
+def _worker_orchestration(rank, world, port, out):
+    """gdelta_fwd_seqshard itself, with its three GPU calls replaced inside this
+    test by float64 oracle stand-ins of the same contract."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import oracle
+    import synth
+    from channel_gated_delta_b200 import seqshard
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    B, H, dk, dv, T = 2, 2, 16, 8, 120
+    inp = synth.generate(synth.GdnShape(B=B, T=T, H=H, dk=dk, dv=dv, dtype="f32", u_low=-4, u_high=0, seed=23))
+    S_in = torch.from_numpy(np.random.Generator(np.random.PCG64(4)).standard_normal((B, H, dk, dv)) * 0.3)
+    bounds = np.linspace(0, T, world + 1).astype(int)
+    seg = _segment(inp, bounds[rank], bounds[rank + 1])
+
+    def fake_fwd(q, k, v, b, w, z, g, log_alpha, gamma_stat=None, S_in=None, y=None, **kw):
+        t = {"q": q, "k": k, "v": v, "b": b, "w": w, "z": z, "g": g, "log_alpha": log_alpha,
+             "gamma_stat": gamma_stat}
+        if t["z"] is None:
+            t["z"] = torch.zeros_like(q)
+        r = oracle.forward_full(t, S0=None if S_in is None else S_in.numpy())
+        return torch.from_numpy(r["y"]), torch.from_numpy(r["S"])
+
+    def fake_map(q, k, v, b, w, z, g, log_alpha, **kw):
+        zero = torch.zeros(q.shape, dtype=q.dtype)
+        eye = torch.eye(dk, dtype=torch.float64).expand(B, H, dk, dk).contiguous()
+        _, A = fake_fwd(q, k, zero, b, zero, None, zero, log_alpha, S_in=eye)
+        _, D = fake_fwd(q, k, v, b, w, None, g, log_alpha)
+        return A, D
+
+    seqshard.gdelta_fwd_chunked = fake_fwd
+    seqshard.gdelta_segment_map = fake_map
+    seqshard.compose_affine = lambda A, S, D: D.clone() if S is None else A @ S + D
+    y, S_final = seqshard.gdelta_fwd_seqshard(seg["q"], seg["k"], seg["v"], seg["b"], seg["w"], seg["z"],
+                                              seg["g"], seg["log_alpha"], gamma_stat=seg["gamma_stat"],
+                                              S_in=S_in)
+    full = oracle.forward_full(inp, S0=S_in.numpy())
+    y_ref = full["y"][:, bounds[rank]:bounds[rank + 1]]
+    out[rank] = (float(np.max(np.abs(y.numpy() - y_ref))), float(np.max(np.abs(S_final.numpy() - full["S"]))))
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_seqshard_forward_orchestration(world):
+    """Every rank's y is its slice of the whole-sequence output and every rank
+    ends with the whole sequence's final state (S_in given, B = H = 2)."""
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_worker_orchestration, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        e_y, e_s = out[r]
+        assert e_y < 1e-9 and e_s < 1e-9, (r, e_y, e_s)
