@@ -46,7 +46,7 @@ static gdelta_status check_fwd(const gdelta_fwd_args *a, bool need_tensors = tru
         if (!a->beta && (!a->b || !a->w)) return GDELTA_ERR_INVALID_ARG;
     }
     const void *ptrs[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->gamma_stat,
-                          a->S_in, a->S_out, a->y, a->o_raw, a->workspace};
+                          a->S_in, a->S_out, a->y, a->o_raw, a->workspace, a->beta};
     for (const void *p : ptrs)
         if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
     return GDELTA_OK;
@@ -211,7 +211,7 @@ gdelta_status gdelta_decode_step(const gdelta_decode_args *a, void *stream) {
     if (!dim_ok(a->dk) || !dim_ok(a->dv)) return GDELTA_ERR_UNSUPPORTED;
     if (!a->q || !a->k || !a->v || !a->g || !a->log_alpha || !a->S || !a->y) return GDELTA_ERR_INVALID_ARG;
     const void *ptrs[] = {a->q, a->k, a->z, a->b, a->v, a->w, a->g, a->log_alpha, a->gamma_stat,
-                          a->S, a->y, a->o_raw};
+                          a->S, a->y, a->o_raw, a->beta};
     for (const void *p : ptrs)
         if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
     DecodeParams p;

@@ -92,6 +92,7 @@ def test_reduced_gate_forms_are_validated_on_the_host(lib):
     assert f(ctypes.byref(_args(decay_per_token=2)), None) == 1
     assert f(ctypes.byref(_args(qk_raw=2)), None) == 1
     assert lib.gdelta_fwd_selected_path(ctypes.byref(_args(beta=beta))) == -1
+    assert f(ctypes.byref(_args(b=None, w=None, beta=beta + 2)), None) == 3     # beta 16-byte aligned too
     # accepted forms: no z; beta alone; beta with a per-token decay
     for kw in ({"z": None}, {"qk_raw": 1}, {"b": None, "w": None, "beta": beta},
                {"b": None, "w": None, "beta": beta, "decay_per_token": 1, "z": None}):
