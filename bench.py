@@ -61,6 +61,10 @@ def parse():
                     help="timed gdelta_bwd calls on the workload (0 = skip the backward measurement)")
     ap.add_argument("--no-forms", action="store_true",
                     help="skip the forward timings of the reduced gate forms")
+    ap.add_argument("--no-gate-proj", action="store_true",
+                    help="skip the five-gate projection timing")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the forward timings of the other full-size workloads (350M layer, 32k tokens)")
     # profiling aid: a smaller case of the same workload (fewer batch rows) for
     # ncu captures that must stay small; the bench line itself uses the default
     ap.add_argument("--batch", type=int, default=0,
@@ -288,6 +292,12 @@ def run_ours(args, rank, local, world):
     # ---- forward alone on the reduced gate forms (same workload shape)
     forms = None if args.no_forms else run_forms(args, gd, d, shape, dev, stream, ws, world)
 
+    # ---- forward alone on the other full-size workloads
+    configs = None if (args.no_configs or args.batch > 0) else run_configs(args, gd, dev, stream, rank, world)
+
+    # ---- the five-gate projection that produces the gates of this layer
+    gproj = None if args.no_gate_proj else run_gate_proj(args, gd, shape, dev, stream, rank, world)
+
     # ---- backward pass on the same workload
     bwd = run_bwd(args, gd, d, shape, dev, stream, world) if args.bwd_calls > 0 else None
 
@@ -347,6 +357,8 @@ def run_ours(args, rank, local, world):
         "clocks": clk,
         "decode": dec,
         "forms": forms,
+        "configs": configs,
+        "gate_proj": gproj,
         "stream": stream_res,
         "backward": bwd,
     }
@@ -366,6 +378,10 @@ def run_decode(args, dev, stream, rank, world):
             for i in range(8)]
     y = torch.empty(B, H, dv, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # Written, the flush buffer would leave up to the whole L2 dirty, and its
+    # write-back would land in the next timed step; reading a second buffer
+    # larger than L2 afterwards writes those lines back before the step.
+    flush_read = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
 
     def one(i):
         t = pool[i % len(pool)]
@@ -379,6 +395,7 @@ def run_decode(args, dev, stream, rank, world):
     barrier(world)
     for i in range(n):
         flush.zero_()                                   # evict the state from L2 (untimed)
+        flush_read.sum()                                # and leave L2 clean (untimed)
         evs[i][0].record(stream)
         one(i)
         evs[i][1].record(stream)
@@ -403,7 +420,8 @@ def run_decode(args, dev, stream, rank, world):
         "roofline": {"bound": "hbm", "kernel": "gdn2_decode_kernel", "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm,
                      "traffic": recorded_traffic("channel_gated_delta_b200/csrc/decode.cu")},
-        "l2": "256 MB buffer written between timed steps (state evicted)",
+        "l2": "between timed steps a 256 MB buffer is written (state evicted), then a second 256 MB "
+              "buffer is read (the first buffer's dirty lines written back before the step)",
         "state_init": "random N(0, 0.05^2) state (timing does not depend on values)",
     }
 
@@ -481,6 +499,111 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
             out[name]["torch_preprocess_then_fwd_ms_median"] = max_over_ranks(
                 statistics.median(a.elapsed_time(c) for a, c in ev2), world)
     return out
+
+
+OTHER_CONFIGS = ("layer350m_bf16", "long32k_bf16")
+
+
+def run_configs(args, gd, dev, stream, rank, world):
+    """gdelta_fwd_chunked alone on the 350M-scale layer (B8 T4096 H8) and the
+    32768-token sequence (B1 T32768 H16), each with its own inputs from
+    ``synth`` (the generators of the parity tests), CUDA events around every
+    call.  Inputs are larger than L2 in both, so no flush."""
+    import synth
+    hbm, kind = peaks()
+    out = {}
+    for name in OTHER_CONFIGS:
+        shape = synth.CONFIGS[name]
+        B, T, H, dk, dv, C = shape.B, shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+        host = synth.generate(shape, seed=shape.seed + 1000 * rank)
+        d = {k: v.to(dev) for k, v in host.items()}
+        del host
+        S = torch.empty(B, H, dk, dv, device=dev)
+        y = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+        nws = gd.gdelta_fwd_workspace_bytes(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"],
+                                            d["log_alpha"], chunk=C, path=args.path)
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+
+        def call():
+            gd.gdelta_fwd_chunked(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"],
+                                  gamma_stat=d["gamma_stat"], S_in=None, S_out=S, y=y, chunk=C,
+                                  path=args.path, workspace=ws, stream=stream)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        if gd.gdelta_get_last_device_error(stream) != 0:
+            raise RuntimeError(f"device status word set during the {name} warm-up")
+        n = max(3, min(args.steps, 10))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        barrier(world)
+        for a, c in evs:
+            a.record(stream)
+            call()
+            c.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
+        nb = fwd_bytes(B, T, H, dk, dv, 2)
+        gbs = nb / (ms * 1e-3) / 1e9
+        out[name] = {
+            "workload": f"{name}: B{B} T{T} H{H} dk=dv={dk} chunk {C}, bf16 tokens, fp32 log-decay and state, "
+                        "S_in = 0",
+            "fwd_ms_median": ms, "tokens_per_s": B * T * world / (ms * 1e-3), "timed_calls": n,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_source": kind, "algorithmic_bytes_per_launch": nb, "launch_ms": ms},
+            "l2": "inputs larger than the 126 MB L2; no flush",
+        }
+        del d, S, y, ws
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_gate_proj(args, gd, shape, dev, stream, rank, world):
+    """gdelta_gate_proj on the Muir 1.34B-scale layer's tokens: N = B*T rows of
+    d = H*128, ranks (64, 64, 128, 128, 128), synthetic weights.  Algorithmic
+    bytes: x and the weights read once, the five gates written once (four bf16,
+    log-decay fp32); FLOPs 4 N d R."""
+    import synth
+    B, T, H, dk = shape.B, shape.T, shape.H, shape.dk
+    N, d = B * T, H * dk
+    ranks = synth.GATE_RANKS
+    R = sum(ranks)
+    inp = {k: v.to(dev) for k, v in synth.gate_proj_inputs(N, d, seed=4 + rank).items()}
+    out = {"log_alpha": torch.empty(N, d, device=dev)}
+    out.update({n: torch.empty(N, d, dtype=torch.bfloat16, device=dev) for n in ("b", "g", "w", "z")})
+    ws = torch.empty(N * 2 * R * 2 + 256, dtype=torch.uint8, device=dev)     # the codes as two bf16 parts
+
+    def call():
+        gd.gdelta_gate_proj(inp["x"], inp["w_down"], inp["w_up"], inp["bias"], ranks=ranks, out=out,
+                            workspace=ws, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    if gd.gdelta_get_last_device_error(stream) != 0:
+        raise RuntimeError("device status word set during the gate projection warm-up")
+    n = max(3, min(args.steps, 20))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier(world)
+    for a, c in evs:
+        a.record(stream)
+        call()
+        c.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
+    nbytes = N * d * 2 + 2 * d * R * 2 + 5 * d * 4 + N * d * (4 * 2 + 4)
+    flops = 4.0 * N * d * R
+    hbm, kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "workload": f"x [{N}, {d}] bf16 (the B{B} T{T} H{H} layer's tokens), ranks {list(ranks)}, synthetic weights",
+        "kernel": "gate_proj_kernel (down: codes = x w_down; up: five grouped products, bias, activations)",
+        "ms_median": ms, "tokens_per_s": N * world / (ms * 1e-3), "timed_calls": n,
+        "algorithmic_bytes": nbytes, "flops": flops, "tflops": flops / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_source": kind,
+                     "note": "4 N d R flops at the measured bf16 peak would take less time than the bytes"},
+    }
 
 
 def bwd_bytes(B, T, H, dk, dv, tok_bytes):

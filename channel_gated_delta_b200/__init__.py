@@ -35,6 +35,9 @@ __all__ = [
     "gdelta_fwd_chunked",
     "gdelta_decode_step",
     "gdelta_bwd",
+    "gdelta_gate_proj",
+    "gdelta_set_wait_limit",
+    "gdelta_set_wait_timeout_test",
     "gdelta_get_last_device_error",
 ]
 
@@ -318,6 +321,66 @@ def gdelta_bwd(q, k, v, b, w, z, g, log_alpha, grad_y, *, gamma_stat=None, S_in=
     a.workspace_bytes = workspace.numel() * workspace.element_size()
     _check(_lib().gdelta_bwd(ctypes.byref(a), _stream(stream)), "gdelta_bwd")
     return out
+
+
+GATE_RANKS = (64, 64, 128, 128, 128)
+
+
+def _gate_proj_struct(x, w_down, w_up, bias, ranks, out, workspace) -> _native.GateProjArgs:
+    if x.dim() != 2:
+        raise ValueError("x must be [N, d]")
+    N, d = x.shape
+    R = int(sum(ranks))
+    a = _native.GateProjArgs()
+    a.N, a.d = int(N), int(d)
+    for i, r in enumerate(ranks):
+        a.ranks[i] = int(r)
+    bf = torch.bfloat16
+    a.x = _dev_ptr(x, "x", bf, (N, d))
+    a.w_down = _dev_ptr(w_down, "w_down", bf, (d, R))
+    a.w_up = _dev_ptr(w_up, "w_up", bf, (R, d))
+    a.bias = _dev_ptr(bias, "bias", torch.float32, (5, d))
+    if out is not None:
+        a.log_alpha = _dev_ptr(out["log_alpha"], "log_alpha", torch.float32, (N, d))
+        for n in ("b", "g", "w", "z"):
+            setattr(a, n, _dev_ptr(out[n], n, bf, (N, d)))
+    if workspace is not None:
+        a.workspace = _dev_ptr(workspace, "workspace")
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    return a
+
+
+def gdelta_gate_proj(x, w_down, w_up, bias, *, ranks=GATE_RANKS, out=None, workspace=None, stream=None) -> dict:
+    """Five-gate low-rank projection (Muir review §2.3): x [N, d] bf16,
+    w_down [d, R], w_up [R, d] bf16 (gate blocks in the order f, b, g, w, q),
+    bias [5, d] fp32.  Returns the mixer's gate inputs as [N, d] tensors:
+    log_alpha (fp32) = log sigmoid(f), b = 2 sigmoid, g, w = sigmoid, z = the
+    q logit (bf16).  ``out`` (a dict with those keys) and ``workspace`` are
+    allocated when not given."""
+    N, d = x.shape
+    if out is None:
+        out = {"log_alpha": torch.empty((N, d), dtype=torch.float32, device=x.device)}
+        out.update({n: torch.empty((N, d), dtype=torch.bfloat16, device=x.device) for n in ("b", "g", "w", "z")})
+    if workspace is None:
+        need = int(_lib().gdelta_gate_proj_workspace_bytes(
+            ctypes.byref(_gate_proj_struct(x, w_down, w_up, bias, ranks, None, None))))
+        if need == 0:
+            raise GdeltaError(2, "gdelta_gate_proj_workspace_bytes")
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    a = _gate_proj_struct(x, w_down, w_up, bias, ranks, out, workspace)
+    _check(_lib().gdelta_gate_proj(ctypes.byref(a), _stream(stream)), "gdelta_gate_proj")
+    return out
+
+
+def gdelta_set_wait_limit(polls: int) -> None:
+    """Polls before a tensor-core kernel's bounded wait gives up (0 = default 2^20)."""
+    _check(_lib().gdelta_set_wait_limit(int(polls)), "gdelta_set_wait_limit")
+
+
+def gdelta_set_wait_timeout_test(on: bool) -> None:
+    """Failure-path test switch: tensor-core forward calls queued while it is on
+    first wait on a barrier nothing completes and report GDELTA_ERR_TIMEOUT."""
+    _check(_lib().gdelta_set_wait_timeout_test(int(bool(on))), "gdelta_set_wait_timeout_test")
 
 
 def gdelta_get_last_device_error(stream=None) -> int:

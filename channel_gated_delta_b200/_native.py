@@ -39,6 +39,10 @@ EXPORTED = (
     "gdelta_decode_step",
     "gdelta_bwd_workspace_bytes",
     "gdelta_bwd",
+    "gdelta_gate_proj_workspace_bytes",
+    "gdelta_gate_proj",
+    "gdelta_set_wait_limit",
+    "gdelta_set_wait_timeout_test",
     "gdelta_get_last_device_error",
 )
 
@@ -86,6 +90,15 @@ class BwdArgs(ctypes.Structure):
     ]
 
 
+class GateProjArgs(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("ranks", ctypes.c_int32 * 5),
+        ("x", _vp), ("w_down", _vp), ("w_up", _vp), ("bias", _fp),
+        ("log_alpha", _fp), ("b", _vp), ("g", _vp), ("w", _vp), ("z", _vp),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _lib = None
 
 
@@ -122,6 +135,14 @@ def load(path: str = LIB_PATH):
     lib.gdelta_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp]
     lib.gdelta_decode_step.restype = ctypes.c_int
     lib.gdelta_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
+    lib.gdelta_gate_proj_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdelta_gate_proj_workspace_bytes.argtypes = [ctypes.POINTER(GateProjArgs)]
+    lib.gdelta_gate_proj.restype = ctypes.c_int
+    lib.gdelta_gate_proj.argtypes = [ctypes.POINTER(GateProjArgs), _vp]
+    lib.gdelta_set_wait_limit.restype = ctypes.c_int
+    lib.gdelta_set_wait_limit.argtypes = [ctypes.c_uint32]
+    lib.gdelta_set_wait_timeout_test.restype = ctypes.c_int
+    lib.gdelta_set_wait_timeout_test.argtypes = [ctypes.c_int32]
     lib.gdelta_get_last_device_error.restype = ctypes.c_int
     lib.gdelta_get_last_device_error.argtypes = [_vp]
     _lib = lib

@@ -57,6 +57,8 @@ struct FwdParams {
     int decay_tok;
     int qk_raw;
     int *status;
+    unsigned wait_limit;     // polls before a bounded wait gives up
+    int stall;               // 1: the kernels first wait on a barrier nothing completes (failure-path tests)
 };
 
 struct DecodeParams {
@@ -84,6 +86,20 @@ struct BwdParams {
     float *ws_ckpt, *ws_chunk, *ws_dgam;
 };
 
+// Five-gate low-rank projection (gdelta.h, gdelta_gate_proj).
+struct GateProjParams {
+    int N, d;
+    int ranks[5];
+    const void *x, *w_down, *w_up;
+    const float *bias;
+    void *codes;             // workspace: [N, R] bf16
+    float *log_alpha;
+    void *b, *g, *w, *z;
+    int *status;
+    unsigned wait_limit;
+    int stall;
+};
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdParams &p, int dtype, cudaStream_t stream);
@@ -97,5 +113,7 @@ cudaError_t launch_state_affine(float *S_out, const float *A, const float *S_in,
 cudaError_t launch_fwd_tc(const FwdParams &p, void *workspace, cudaStream_t stream);
 size_t fwd_tc_workspace_bytes(int B, int H, int T);
 bool fwd_tc_supported(int dtype, int dk, int dv, int chunk);
+size_t gate_proj_workspace_bytes(int N, int R);
+cudaError_t launch_gate_proj(const GateProjParams &p, cudaStream_t stream);
 
 }  // namespace gdelta

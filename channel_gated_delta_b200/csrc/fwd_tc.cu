@@ -132,6 +132,13 @@ constexpr int kWinANAB = kWinBP + 128 * 256;  // [N ; Aq ; Bq]   192 x 64
 constexpr int kWinVH = kWinANAB + 192 * 128;  // V^               64 x 128
 constexpr int kWinVEC = kWinVH + 64 * 256;    // e^c, e^{Lambda_{n-1} - c}
 constexpr int kWinBytes = kWinVEC + 1024;
+static_assert(kWinVH % 32 == 0, "the shared tiles split into two 16-byte-multiple halves");
+#ifndef GDN2_REC_PREFETCH
+#define GDN2_REC_PREFETCH 4
+#endif
+// The chain kernel copies a window's record two windows ahead and prefetches
+// the record this many windows ahead into L2 (0 = no prefetch).
+constexpr int kRecPrefetch = GDN2_REC_PREFETCH;
 
 // Chain-kernel TMEM columns
 constexpr uint32_t kTmP = 0;       // shorter chunks: P (128 x 128)
@@ -156,7 +163,14 @@ struct TcParams {
     int decay_tok;               // 1: la holds one log-decay per token and head
     int qk_raw;                  // 1: q and k need SiLU and l2 normalisation
     int NW;                  // windows of 64 tokens per head
+    uint32_t spin;           // polls before a bounded wait on another party gives up
+    int stall;               // 1: wait first on a barrier nothing completes, so that the wait runs out
 };
+
+// Polls of a wait for this CTA's own asynchronous work (bulk copies, MMAs)
+// before the CTA leaves or frees TMEM: independent of the configurable limit,
+// so that a small limit never lets a CTA exit with a copy or MMA in flight.
+constexpr uint32_t kDrainPolls = 1u << 22;
 
 __device__ __forceinline__ void bf16x8_to_f(const uint4 &u, float *f) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -292,6 +306,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     const uint32_t s_mbar = tc::smem_u32(mbar), s_rbar = s_mbar + 8, s_xbar = s_mbar + 24;
     const uint32_t s_ibar = s_mbar + 40, s_obar = s_mbar + 56, s_fbar = s_mbar + 72;
     const uint32_t s_lq = s_mbar + 144, s_lfree = s_mbar + 160;  // record request posted / slot read
+    const uint32_t s_stall = s_mbar + 192;                         // never completed (failure-path tests)
     const uint32_t peer_rank = crank ^ 1u;
     const uint32_t r_peer = tc::mapa(tc::smem_u32(peer), peer_rank);
     const uint32_t r_pflag = tc::mapa(tc::smem_u32(pflag), peer_rank);
@@ -306,6 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     if (tid == 0) {
         for (int i = 0; i < 11; ++i) tc::mbar_init(s_mbar + 8 * i, 1);
         for (int i = 0; i < 4; ++i) tc::mbar_init(s_lq + 8 * i, 1);
+        tc::mbar_init(s_stall, 1);
         tc::mbar_arrive_expect_tx(s_xbar, 65 * 4);   // the peer's sums of chunk 0 (64 rows and a flag)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
@@ -332,6 +348,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     // fence: a thread that has bulk copies in flight and then fences the async
     // proxy (as the state warps do after staging operand tiles) waits for those
     // copies, which would tie every window to the record two windows ahead.
+    // Window wp's record into L2; the two CTAs of the cluster split the shared
+    // tiles between them and each fetches its own half of V^.
+    auto prefetch_rec = [&](int wp) {
+        const uint8_t *pf = p.ws + (wbase + wp) * kWinBytes;
+        const uint32_t half = (uint32_t)kWinVH / 2;
+        tc::bulk_prefetch_l2(pf + crank * half, half);
+        tc::bulk_prefetch_l2(pf + kWinVH + crank * (64 * 128), 64 * 128);
+        if (crank == 0) tc::bulk_prefetch_l2(pf + kWinVEC, 2 * 128 * 4);
+    };
     auto issue_rec = [&](int w, int b) {         // window w's record -> buffer b
         const uint8_t *rec = p.ws + (wbase + w) * kWinBytes;
         uint8_t *dst = sm + b * L::BUF;
@@ -342,13 +367,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         tc::bulk_g2s(tc::smem_u32(dst + L::ANAB), rec + kWinANAB, 192 * 128, bar);
         tc::bulk_g2s(tc::smem_u32(dst + L::VH), rec + kWinVH + crank * (64 * 128), 64 * 128, bar);
         tc::bulk_g2s(tc::smem_u32(dst + L::EV), rec + kWinVEC, 2 * 128 * 4, bar);
+        // the record kRecPrefetch windows further on is brought into L2 now, so that
+        // its copy into shared memory is served from L2 instead of DRAM (the first
+        // two copies also cover the windows before that distance)
+        if (kRecPrefetch > 2) {
+            for (int wp = (w < 2 ? w + 2 : w + kRecPrefetch); wp <= w + kRecPrefetch; wp += 2)
+                if (wp < NW) prefetch_rec(wp);
+        }
     };
     static_assert(L::BUF == 2 * 128 * 256 + 192 * 128 + 64 * 128 + 1024, "record buffer = bytes of one record copy");
 
+    int mma_pending = -1;                         // parity of an MMA commit whose wait ran out
     if (warp < 8) {
-        // Wait for the MMAs committed so far; a timeout marks a local abort.
+        // Wait for the MMAs committed so far; a timeout marks a local abort (the
+        // commit is drained before TMEM is freed).
         auto wait_mma = [&]() -> bool {
-            if (!tc::mbar_wait(s_mbar, phase)) flags[0] = 1;
+            if (!tc::mbar_wait(s_mbar, phase, p.spin)) {
+                flags[0] = 1;
+                mma_pending = (int)phase;
+            }
             phase ^= 1u;
             main_sync();
             tc::fence_after_sync();
@@ -360,15 +397,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         uint32_t nreq = 0;
         auto enqueue = [&](int w, int b) {
             const uint32_t k = nreq++, sl = k & 1u;
-            if (k >= 2 && !tc::mbar_wait(s_lfree + 8u * sl, ((k >> 1) - 1) & 1u)) flags[0] = 1;
+            if (k >= 2 && !tc::mbar_wait(s_lfree + 8u * sl, ((k >> 1) - 1) & 1u, p.spin)) flags[0] = 1;
             req[2 * sl] = w;
             req[2 * sl + 1] = b;
             tc::mbar_arrive_local(s_lq + 8u * sl);
         };
 
+        // failure-path test: a wait that nothing completes runs out before any work is issued
+        if (p.stall) {
+            if (tid == 0 && !tc::mbar_wait(s_stall, 0, p.spin)) flags[0] = 1;
+            main_sync();
+        }
         int loaded[2] = {-1, -1};                     // window whose record buffer b holds or receives
         bool inflight[2] = {false, false};            // a copy into buffer b not yet waited for
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < 2 && flags[0] == 0; ++b)
             if (win_fast(b)) {
                 if (tid == 0) enqueue(b, b);
                 loaded[b] = b;
@@ -393,13 +435,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             // an abort agreed by the readout warps becomes this group's abort at the barrier below
             if (tid == 0 && flags[3] != 0) flags[0] = 1;
             if (fast) {
-                if (!tc::mbar_wait(s_rbar + 8u * B, rphase[B])) flags[0] = 1;
+                if (!tc::mbar_wait(s_rbar + 8u * B, rphase[B], p.spin)) flags[0] = 1;
                 rphase[B] ^= 1u;
                 inflight[B] = false;
             } else if (inflight[B ^ 1]) {
                 // the other buffer is this window's scratch: a record arriving there
                 // lands first, and is copied again after the window
-                if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), rphase[B ^ 1])) flags[0] = 1;
+                if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), rphase[B ^ 1], p.spin)) flags[0] = 1;
                 rphase[B ^ 1] ^= 1u;
                 inflight[B ^ 1] = false;
             }
@@ -785,7 +827,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     // ---- I: [R; O] = [W'; Qp] S_c + [N; Aq] V^ ;  X += Kc^T V^
                     if (tid == 0) {
                         // the slot's previous O has been read out of TMEM (and its chunk info)
-                        if (uses[slot] > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u)) flags[0] = 1;
+                        if (uses[slot] > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u, p.spin))
+                            flags[0] = 1;
                         // the readout warps learn the chunk's tokens now (to fetch the gate early)
                         info[4 * slot] = t0;
                         info[4 * slot + 1] = n;
@@ -873,14 +916,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         // no more chunks: tell the readout warps
         if (tid == 0) {
             const uint32_t slot = (uint32_t)(chunk & 1);
-            if (uses[slot] > 0) tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u);
+            if (uses[slot] > 0) tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u, p.spin);
             info[4 * slot + 2] = 1;
             tc::mbar_arrive_local(s_ibar + 8u * slot);
         }
         if (tid == 0) enqueue(-1, 0);
         // copies still in flight (the loop ended early) complete before exit
         for (int b = 0; b < 2; ++b)
-            if (inflight[b]) tc::mbar_wait(s_rbar + 8u * b, rphase[b]);
+            if (inflight[b]) tc::mbar_wait(s_rbar + 8u * b, rphase[b], kDrainPolls);
 
         // ---- S_out = Diag(fprev) X
         if (flags[0] == 0 && p.S_out && T > 0) {
@@ -901,7 +944,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 const uint32_t sl = k & 1u;
                 bool got = false;
                 for (int tries = 0; tries < 64 && !got; ++tries) {
-                    got = tc::mbar_wait(s_lq + 8u * sl, (k >> 1) & 1u);
+                    got = tc::mbar_wait(s_lq + 8u * sl, (k >> 1) & 1u, p.spin);
                     if (!got && (flags[0] != 0 || flags[3] != 0)) break;
                 }
                 if (!got) break;
@@ -918,7 +961,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         for (int c = 0;; ++c) {
             const uint32_t slot = (uint32_t)(c & 1), ph = (uint32_t)(c >> 1) & 1u;
             // one thread waits, the barrier hands its view (and the chunk info) to the rest
-            if (et == 0 && !tc::mbar_wait(s_ibar + 8u * slot, ph)) flags[3] = 1;
+            if (et == 0 && !tc::mbar_wait(s_ibar + 8u * slot, ph, p.spin)) flags[3] = 1;
             asm volatile("bar.sync 3, 64;" ::: "memory");
             if (flags[3] != 0) break;
             // every row is done with the previous chunk's exchange slot: it now
@@ -947,7 +990,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 }
             }
             bool ok = true;
-            if (et == 0) ok = tc::mbar_wait(s_obar + 8u * slot, ph);
+            if (et == 0) ok = tc::mbar_wait(s_obar + 8u * slot, ph, p.spin);
             asm volatile("bar.sync 3, 64;" ::: "memory");
             tc::fence_after_sync();
             float ov[2][32];
@@ -968,7 +1011,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             tc::st_async_f32(r_peer + slot * 256u + 4u * et, ss, r_xbar + 8u * slot);
             if (et == 0) tc::st_async_s32(r_pflag + 4u * slot, (ok && flags[0] == 0) ? 0 : 1, r_xbar + 8u * slot);
             if (et == 0) {
-                const bool got = tc::mbar_wait_cluster(s_xbar + 8u * slot, ph);
+                const bool got = tc::mbar_wait_cluster(s_xbar + 8u * slot, ph, p.spin);
                 if (!got || pflag[slot] != 0 || !ok) flags[3] = 1;
             }
             asm volatile("bar.sync 3, 64;" ::: "memory");
@@ -1016,6 +1059,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     __syncthreads();
     if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
     if ((flags[0] != 0 || flags[3] != 0) && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
+    // an MMA whose completion wait ran out finishes before its TMEM is freed
+    if (tid == 0 && mma_pending >= 0) tc::mbar_wait(s_mbar, (uint32_t)mma_pending, kDrainPolls);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
     // no CTA leaves while its peer may still write into its shared memory
     tc::cluster_sync();
@@ -1031,19 +1079,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
 // chain kernel in shorter chunks.
 // ---------------------------------------------------------------------------
 namespace {
+// 74.8 KB, so that three CTAs share an SM.  Regions are reused as the window
+// proceeds: after P, the [Kc; K^c] tile (bulk-copied to the record) holds the
+// fp32 L / T^-1, the merge buffer and the fp16 T^-1 tile; after the operand
+// build, the scan scratch holds the fp16 M tile.
 struct IntraSmem {
-    static constexpr int AP = 0;                  // [Kp ; Qp]   128 x 128 fp16
-    static constexpr int BP = AP + 128 * 256;     // [Kc ; K^c]  128 x 128; after P: fp32 L / T^-1 + merge buffer
-    static constexpr int TI = BP + 128 * 256;     // T^-1         64 x 64
-    static constexpr int MM = TI + 64 * 128;      // M            64 x 64
-    static constexpr int WT = MM + 64 * 128;      // fp32 per-warp log-decay totals [8][128]
-    static constexpr int PR = WT + 8 * 128 * 4;   // fp32 Lambda at the probe tokens [8][128]
-    static constexpr int VEC = PR + 8 * 128 * 4;  // gamma_stat, exact diagonals, span maxima
-    static constexpr int MISC = VEC + 512 * 4;    // mbarrier, TMEM slot, flags
+    static constexpr int AP = 0;                  // [Kp ; Qp]   128 x 128 fp16 (then W' over Kp, Aq/Bq over Qp)
+    static constexpr int BP = AP + 128 * 256;     // [Kc ; K^c]  128 x 128
+    static constexpr int LW = BP;                 //   after P: fp32 L, then T^-1   [64][kLW]
+    static constexpr int YB = LW + 64 * kLW * 4;  //   merge buffer                 [32][kYS]
+    static constexpr int TI = BP + 23 * 1024;     //   T^-1, 64 x 64 fp16 (1024-byte aligned)
+    static constexpr int SCR = BP + 128 * 256;    // scan scratch, then M (64 x 64 fp16)
+    static constexpr int WT = SCR;                //   fp32 per-warp log-decay totals [8][128]
+    static constexpr int PR = WT + 8 * 128 * 4;   //   fp32 Lambda of tokens 0 and 63 [2][128]
+    static constexpr int MM = SCR;
+    static constexpr int VEC = SCR + 64 * 128;    // gamma_stat [128], exact diagonals [2][64], span maxima [8]
+    static constexpr int MISC = VEC + (128 + 128 + 8) * 4;   // mbarriers, TMEM slot, flags
     static constexpr int TOTAL = MISC + 64;
 };
-constexpr uint32_t kItmW = 0;      // W' (M=64) reuses the columns of P after its epilogue
-constexpr uint32_t kItmN = 128;    // N  (M=64)
+static_assert(IntraSmem::YB + 32 * kYS * 4 <= IntraSmem::TI, "merge buffer before the T^-1 tile");
+static_assert(IntraSmem::TI + 64 * 128 <= IntraSmem::SCR, "T^-1 tile inside the [Kc; K^c] region");
+static_assert(IntraSmem::PR + 2 * 128 * 4 <= IntraSmem::VEC, "scan scratch inside the M region");
+static_assert(3 * (IntraSmem::TOTAL + 1024 + 1024) <= 228 * 1024, "three CTAs per SM");
+// TMEM (128 columns): P (M = 128) at column 0; after its epilogue W' (M = 64)
+// in lanes 0-15 of each 32-lane quadrant and N (M = 64) in lanes 16-31, both
+// from column 0.
+constexpr uint32_t kItmW = 0;
+constexpr uint32_t kItmN = 16u << 16;
 }  // namespace
 
 // Input forms, fixed at compile time: kNoZ reads no z (2 sigmoid(z) = 1), kBeta
@@ -1051,7 +1113,7 @@ constexpr uint32_t kItmN = 128;    // N  (M=64)
 // token and head, kRaw applies SiLU and l2 normalisation to q and k.  All false
 // is the per-channel GDN-2 form on preprocessed q and k.
 template <bool kNoZ, bool kBeta, bool kTok, bool kRaw>
-__global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
+__global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
     using L = IntraSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1063,8 +1125,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
     const int t0 = kC * win, wend = min(T, t0 + kC);
     uint8_t *rec = ws + (size_t)wi * kWinBytes;
 
-    float *lw = (float *)(sm + L::BP);
-    float *yb = lw + 64 * kLW;
+    float *lw = (float *)(sm + L::LW);
+    float *yb = (float *)(sm + L::YB);
     float *wtot = (float *)(sm + L::WT);
     float *probe = (float *)(sm + L::PR);
     float *vec = (float *)(sm + L::VEC);
@@ -1072,18 +1134,23 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
     uint64_t *mbar = (uint64_t *)(sm + L::MISC);
     uint32_t *tslot = (uint32_t *)(sm + L::MISC + 8);
     int *flags = (int *)(sm + L::MISC + 16);
+    const uint32_t s_stall = tc::smem_u32(sm + L::MISC + 32);    // never completed (failure-path tests)
     const uint32_t s_ap = tc::smem_u32(sm + L::AP), s_bp = tc::smem_u32(sm + L::BP);
     const uint32_t s_ti = tc::smem_u32(sm + L::TI), s_mm = tc::smem_u32(sm + L::MM);
     const uint32_t s_mbar = tc::smem_u32(mbar);
 
     if (warp == 0) {
-        tc::tmem_alloc(tc::smem_u32(tslot), 256);
+        tc::tmem_alloc(tc::smem_u32(tslot), 128);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
         tc::mbar_init(s_mbar, 1);
+        tc::mbar_init(s_stall, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
+        // until its record is complete the window is marked for the chain kernel to
+        // process itself, so an abandoned record is never read
+        wflags[wi] = 1;
     }
     if (tid < kDK) gsv[tid] = p.gs ? p.gs[(size_t)h * kDK + tid] : 1.f;
     tc::fence_before_sync();
@@ -1095,9 +1162,13 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
     const int row = 32 * (warp & 3) + lane;
     const int colhalf = warp >> 2;
     float range_max = 0.f;
+    int mma_pending = -1;                         // parity of an MMA commit whose wait ran out
     auto wait_mma = [&]() -> bool {
-        const bool ok = tc::mbar_wait(s_mbar, phase);
-        if (!ok) flags[0] = 1;
+        const bool ok = tc::mbar_wait(s_mbar, phase, p.spin);
+        if (!ok) {
+            flags[0] = 1;
+            mma_pending = (int)phase;
+        }
         phase ^= 1u;
         __syncthreads();
         tc::fence_after_sync();
@@ -1105,52 +1176,65 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
     };
 
     do {
-        // ---- loads (whole 256-byte token rows per instruction) and the log-decay
-        // scan, in log2 units (Lambda * log2 e) so that every decay factor is one ex2
+        // failure-path test: a wait that nothing completes runs out before any work is issued
+        if (p.stall) {
+            if (tid == 0 && !tc::mbar_wait(s_stall, 0, p.spin)) flags[0] = 1;
+            __syncthreads();
+            if (flags[0] != 0) break;
+        }
+        // ---- the log-decay scan, in log2 units (Lambda * log2 e) so that every decay
+        // factor is one ex2.  Warp w owns tokens [8w, 8w+8), lane l channels [4l, 4l+4)
+        // (whole 256-byte token rows per load instruction).  Pass 1 sums the warp's
+        // log-decays for the cross-warp prefix; the build below reads them again token
+        // by token (from L2) and keeps only a running sum, so that a thread never holds
+        // more than two tokens' inputs.
         const int tb = 8 * warp, c4 = 4 * lane;
-        float la[8][4];
-        uint2 kq[8][4];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = tb + u;
-            const bool in = t0 + t < wend;
-            const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gk = gt * kDK + c4;
+        auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
+        auto load_la = [&](int u) -> float4 {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (in) {
+            if (t0 + tb + u < wend) {
                 if (kTok) {
-                    const float s = __ldg(p.la + gt);
-                    x = make_float4(s, s, s, s);
+                    const float sc = __ldg(p.la + gt_of(u));
+                    x = make_float4(sc, sc, sc, sc);
                 } else {
-                    x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                    x = __ldg(reinterpret_cast<const float4 *>(p.la + gt_of(u) * kDK + c4));
                 }
             }
-            la[u][0] = x.x * kLog2e; la[u][1] = x.y * kLog2e; la[u][2] = x.z * kLog2e; la[u][3] = x.w * kLog2e;
-            kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
-            kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-            kq[u][2] = in && !kNoZ ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-            kq[u][3] = !in ? make_uint2(0, 0)
-                      : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
-        }
-#pragma unroll
-        for (int u = 1; u < 8; ++u)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) la[u][c] += la[u - 1][c];
-        *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
-        __syncthreads();
+            return x;
+        };
+        // token u's k, q, z and b (4 bf16 each; zeros past the end of the sequence)
+        auto load_kq = [&](int u, uint2 (&o)[4]) {
+            const bool in = t0 + tb + u < wend;
+            const size_t gt = gt_of(u), gk = gt * kDK + c4;
+            o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
+            o[1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
+            o[2] = in && !kNoZ ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+            o[3] = !in ? make_uint2(0, 0)
+                  : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
+        };
+        float off[4] = {0.f, 0.f, 0.f, 0.f};
         {
-            float off[4] = {0.f, 0.f, 0.f, 0.f};
+            float tot[4] = {0.f, 0.f, 0.f, 0.f}, first[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 x = load_la(u);
+                if (u == 0) {
+                    first[0] = x.x * kLog2e; first[1] = x.y * kLog2e; first[2] = x.z * kLog2e; first[3] = x.w * kLog2e;
+                }
+                tot[0] += x.x * kLog2e; tot[1] += x.y * kLog2e; tot[2] += x.z * kLog2e; tot[3] += x.w * kLog2e;
+            }
+            *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(tot[0], tot[1], tot[2], tot[3]);
+            __syncthreads();
             for (int ww = 0; ww < warp; ++ww) {
                 const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
                 off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) la[u][c] += off[c];
+            // Lambda at token 0 and at the last token (zero-padded log-decay past the end)
+            if (warp == 0) *reinterpret_cast<float4 *>(probe + c4) = make_float4(first[0], first[1], first[2], first[3]);
+            if (warp == 7)
+                *reinterpret_cast<float4 *>(probe + kDK + c4) =
+                    make_float4(off[0] + tot[0], off[1] + tot[1], off[2] + tot[2], off[3] + tot[3]);
         }
-        // Lambda at token 0 and at the last token (zero-padded log-decay past the end)
-        if (warp == 0) *reinterpret_cast<float4 *>(probe + c4) = make_float4(la[0][0], la[0][1], la[0][2], la[0][3]);
-        if (warp == 7) *reinterpret_cast<float4 *>(probe + kDK + c4) = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
         __syncthreads();
         const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
         const float4 ln4 = *reinterpret_cast<const float4 *>(probe + kDK + c4);
@@ -1174,6 +1258,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
 
         // ---- operand tiles: P operands to shared memory (Qp, Kc and K^c reach the
         // record from there by bulk copy); the pivot vectors straight to the record
+        uint2 vw_nx[2];                               // token 0's v and w, loaded during the build
         {
             const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
             const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
@@ -1189,17 +1274,35 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 rv[32 + lane] = make_float4(ex2(lnv[0] - cpiv[0]), ex2(lnv[1] - cpiv[1]), ex2(lnv[2] - cpiv[2]),
                                             ex2(lnv[3] - cpiv[3]));
             }
+            float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
+            float4 la_nx = load_la(0);
+            uint2 kq_nx[4];
+            load_kq(0, kq_nx);
             float dg[16];                             // [u]: q~.k, [8+u]: q~.(b*k) of token tb+u, this lane's channels
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = tb + u;
                 const bool live = t < n;
+                const float4 la_c = la_nx;
+                const uint2 kq_c[4] = {kq_nx[0], kq_nx[1], kq_nx[2], kq_nx[3]};
+                if (u + 1 < 8) {                      // the next token's inputs are in flight meanwhile
+                    la_nx = load_la(u + 1);
+                    load_kq(u + 1, kq_nx);
+                } else {
+                    const bool in = t0 + tb < wend;   // the value side of token 0, for after the build
+                    const size_t gt = gt_of(0), gv = gt * kDV + c4;
+                    vw_nx[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+                    vw_nx[1] = !in ? make_uint2(0, 0)
+                               : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                }
+                lam_run[0] += la_c.x * kLog2e; lam_run[1] += la_c.y * kLog2e;
+                lam_run[2] += la_c.z * kLog2e; lam_run[3] += la_c.w * kLog2e;
                 float kk[4], qq[4], zz[4], bv[4];
                 {
-                    const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][0]);
-                    const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][1]);
-                    const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][2]);
-                    const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][3]);
+                    const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[0]);
+                    const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[1]);
+                    const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[2]);
+                    const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[3]);
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         float2 f;
@@ -1217,7 +1320,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 float dq = 0.f, db = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float lam = live ? la[u][c] : lnv[c];
+                    const float lam = live ? lam_run[c] : lnv[c];
                     const float d = lam - cpiv[c];
                     const float ep = ex2(d), em = ex2(-d);
                     const float kv = live ? kk[c] : 0.f;
@@ -1244,23 +1347,12 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
                 *(uint2 *)(sm + L::BP + off_t) = ukc;
                 *(uint2 *)(sm + L::BP + off_b) = ukh;
             }
-            // the exact diagonals q~_t.k_t and q~_t.(b*k)_t of Aq / Bq
+        // the exact diagonals q~_t.k_t and q~_t.(b*k)_t of Aq / Bq
             const float dsum = reduce_scatter16(dg, lane);
             if ((lane & 1) == 0) {
                 const int vi = (lane >> 1) & 15;
                 (vi < 8 ? diagq : diagb)[tb + (vi & 7)] = dsum;
             }
-        }
-        // value side: loads issued now, consumed while the P product runs
-        uint2 vw[8][2];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = tb + u;
-            const bool in = t0 + t < wend;
-            const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gv = gt * kDV + c4;
-            vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-            vw[u][1] = !in ? make_uint2(0, 0)
-                      : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
         }
         tc::fence_proxy_async();
         __syncthreads();
@@ -1278,12 +1370,21 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             tc::bulk_s2g(rec + kWinAP + 128 * 128 + 64 * 128, s_ap + 128 * 128 + 64 * 128, 64 * 128);  // columns 64-127
             tc::bulk_commit();
         }
-        // V^ = w*v -> window record (the identity padding past n is zero)
+        // V^ = w*v -> window record (the identity padding past n is zero), token by
+        // token with the next token's v and w in flight, while the P product runs
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int t = tb + u;
-            const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
-            const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
+            const uint2 vw_c[2] = {vw_nx[0], vw_nx[1]};
+            if (u + 1 < 8) {
+                const bool in = t0 + t + 1 < wend;
+                const size_t gt = gt_of(u + 1), gv = gt * kDV + c4;
+                vw_nx[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+                vw_nx[1] = !in ? make_uint2(0, 0)
+                           : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+            }
+            const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
+            const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
             float vh[4];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -1305,36 +1406,35 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
             const int t = row & 63;
             const bool upper = row < 64;
             const int tb2 = warp & 1;
-            float v[2][32];
-            tc::tmem_ld32x2(tmem + lane_base + 64 * colhalf, tmem + lane_base + 64 * colhalf + 32, v[0], v[1]);
-            // all warps have read P and the bulk copies have read BP and the Qp rows:
-            // both may now be overwritten
+            // the bulk copies have read BP and the Qp rows: both may now be overwritten
+            // (P stays in TMEM until the W' / N products, issued after a later barrier)
             if (tid == 0) tc::bulk_wait_read();
-            tc::fence_before_sync();
             __syncthreads();
             const float dv_t = upper ? 0.f : (colhalf == 0 ? diagq[t] : diagb[t]);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + 64 * colhalf + 32 * hf, v);
                 if (hf > tb2) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[hf][i] = 0.f;
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
                 } else if (hf == tb2) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const bool keep = upper ? (i < lane) : (i <= lane);
-                        if (!keep) v[hf][i] = 0.f;
-                        if (!upper && i == lane) v[hf][i] = dv_t;
+                        if (!keep) v[i] = 0.f;
+                        if (!upper && i == lane) v[i] = dv_t;
                     }
                 }
                 if (upper && colhalf == 1) {
                     float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(v[hf][4 * q], v[hf][4 * q + 1], v[hf][4 * q + 2], v[hf][4 * q + 3]);
+                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                 } else if (upper) {
-                    store_row32(sm + L::MM, 64, t, 32 * hf, v[hf]);
+                    store_row32(sm + L::MM, 64, t, 32 * hf, v);
                 } else {
-                    store_row32(sm + L::AP + (colhalf == 0 ? 64 * 128 : 128 * 128 + 64 * 128), 64, t, 32 * hf, v[hf]);
+                    store_row32(sm + L::AP + (colhalf == 0 ? 64 * 128 : 128 * 128 + 64 * 128), 64, t, 32 * hf, v);
                 }
             }
         }
@@ -1402,25 +1502,24 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
         if (!wait_mma()) break;
 
         // ---- W' -> staged over Kp (rows 0-63 of AP), N -> over M; both copied to
-        // rows 0-63 of the record's [W'; Qp] and [N; Aq; Bq]
+        // rows 0-63 of the record's [W'; Qp] and [N; Aq; Bq].  One load gives a warp
+        // W' rows in its lanes 0-15 and N rows in lanes 16-31 (N has 64 columns, so
+        // only the warps of the first column half keep those).
         {
-            const int t = 16 * (warp & 3) + lane;
-            const bool valid = lane < 16;
-            float v[2][32];
-            tc::tmem_ld32x2(tmem + lane_base + kItmW + 64 * colhalf, tmem + lane_base + kItmW + 64 * colhalf + 32, v[0],
-                            v[1]);
-            if (valid) {
+            const int t = 16 * (warp & 3) + (lane & 15);
+            const bool nrow = lane >= 16;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    range_max = fmaxf(range_max, maxabs(v[hf], 32));
-                    store_row32(sm + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int col = 64 * colhalf + 32 * hf;
+                float v[32];
+                tc::tmem_ld32(tmem + lane_base + col, v);
+                if (!nrow) {
+                    range_max = fmaxf(range_max, maxabs(v, 32));
+                    store_row32(sm + L::AP, 128, t, col, v);
+                } else if (colhalf == 0) {
+                    range_max = fmaxf(range_max, maxabs(v, 32));
+                    store_row32(sm + L::MM, 64, t, 32 * hf, v);
                 }
-            }
-            float nv[32];
-            tc::tmem_ld32(tmem + lane_base + kItmN + 32 * colhalf, nv);
-            if (valid) {
-                range_max = fmaxf(range_max, maxabs(nv, 32));
-                store_row32(sm + L::MM, 64, t, 32 * colhalf, nv);
             }
         }
         tc::fence_proxy_async();
@@ -1438,9 +1537,11 @@ __global__ void __launch_bounds__(kThreads, 2) gdn2_chunk_intra_tc_kernel(TcPara
 
     if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
     if (flags[0] != 0 && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
+    // an MMA whose completion wait ran out finishes before its TMEM is freed
+    if (tid == 0 && mma_pending >= 0) tc::mbar_wait(s_mbar, (uint32_t)mma_pending, kDrainPolls);
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 256);
+    if (warp == 0) tc::tmem_dealloc(tmem, 128);
 }
 
 size_t fwd_tc_workspace_bytes(int B, int H, int T) {
@@ -1462,6 +1563,8 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.beta = (const __nv_bfloat16 *)fp.beta; p.decay_tok = fp.decay_tok; p.qk_raw = fp.qk_raw;
     p.y = (__nv_bfloat16 *)fp.y; p.o_raw = fp.o_raw; p.eps = fp.eps; p.status = fp.status;
     p.NW = (fp.T + kC - 1) / kC;
+    p.spin = fp.wait_limit;
+    p.stall = fp.stall;
     const size_t nwin = (size_t)fp.B * fp.H * p.NW;
     uint8_t *ws = (uint8_t *)workspace;
     int *wflags = (int *)(ws + nwin * kWinBytes);

@@ -1,5 +1,6 @@
 // C ABI entry points: argument checks on the host, then kernel launches on the
 // caller's stream.  Nothing here allocates device memory.
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -24,6 +25,12 @@ static int *status_ptr() {
     }
     return ptrs[dev];
 }
+
+// Bounded-wait limit of the tensor-core kernels and the failure-path test
+// switch (gdelta_set_wait_limit, gdelta_set_wait_timeout_test).
+constexpr uint32_t kDefaultWaitPolls = 1u << 20;
+static std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
+static std::atomic<int> g_stall_test{0};
 
 static bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
 static bool dim_ok(int d) { return d == 64 || d == 128; }
@@ -189,6 +196,8 @@ gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *a, void *stream) {
     p.y = a->y; p.o_raw = a->o_raw; p.eps = a->eps;
     p.beta = a->beta; p.decay_tok = a->decay_per_token; p.qk_raw = a->qk_raw;
     p.status = status_ptr();
+    p.wait_limit = g_wait_polls.load(std::memory_order_relaxed);
+    p.stall = g_stall_test.load(std::memory_order_relaxed);
     if (path == GDELTA_PATH_TC) {
         p.C = 64;
         const size_t need = fwd_tc_workspace_bytes(a->B, a->H, a->T);
@@ -222,6 +231,63 @@ gdelta_status gdelta_decode_step(const gdelta_decode_args *a, void *stream) {
     p.beta = a->beta; p.decay_tok = a->decay_per_token; p.qk_raw = a->qk_raw;
     return launch_decode(p, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
                                                                            : GDELTA_ERR_CUDA;
+}
+
+static gdelta_status check_gate_proj(const gdelta_gate_proj_args *a, int *R) {
+    if (!a) return GDELTA_ERR_INVALID_ARG;
+    if (a->N < 1 || a->d < 256) return GDELTA_ERR_INVALID_ARG;
+    if (a->d % 256 != 0) return GDELTA_ERR_UNSUPPORTED;
+    int r = 0;
+    for (int i = 0; i < 5; ++i) {
+        if (a->ranks[i] < 64 || a->ranks[i] % 64 != 0) return GDELTA_ERR_UNSUPPORTED;
+        r += a->ranks[i];
+    }
+    if (r % 256 != 0 || r > 2048) return GDELTA_ERR_UNSUPPORTED;
+    *R = r;
+    return GDELTA_OK;
+}
+
+size_t gdelta_gate_proj_workspace_bytes(const gdelta_gate_proj_args *a) {
+    int R = 0;
+    if (check_gate_proj(a, &R) != GDELTA_OK) return 0;
+    return gate_proj_workspace_bytes(a->N, R);
+}
+
+gdelta_status gdelta_gate_proj(const gdelta_gate_proj_args *a, void *stream) {
+    int R = 0;
+    const gdelta_status st = check_gate_proj(a, &R);
+    if (st != GDELTA_OK) return st;
+    const void *req[] = {a->x, a->w_down, a->w_up, a->bias, a->log_alpha, a->b, a->g, a->w, a->z};
+    for (const void *p : req)
+        if (!p) return GDELTA_ERR_INVALID_ARG;
+    const void *ptrs[] = {a->x, a->w_down, a->w_up, a->bias, a->log_alpha, a->b, a->g, a->w, a->z, a->workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDELTA_ERR_ALIGNMENT;
+    if (!a->workspace || a->workspace_bytes < gate_proj_workspace_bytes(a->N, R)) return GDELTA_ERR_WORKSPACE;
+    GateProjParams p{};
+    p.N = a->N;
+    p.d = a->d;
+    for (int i = 0; i < 5; ++i) p.ranks[i] = a->ranks[i];
+    p.x = a->x; p.w_down = a->w_down; p.w_up = a->w_up; p.bias = a->bias;
+    p.codes = a->workspace;
+    p.log_alpha = a->log_alpha; p.b = a->b; p.g = a->g; p.w = a->w; p.z = a->z;
+    p.status = status_ptr();
+    p.wait_limit = g_wait_polls.load(std::memory_order_relaxed);
+    p.stall = g_stall_test.load(std::memory_order_relaxed);
+    const cudaError_t e = launch_gate_proj(p, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue) return GDELTA_ERR_UNSUPPORTED;     // a tensor map was refused
+    return e == cudaSuccess ? GDELTA_OK : GDELTA_ERR_CUDA;
+}
+
+gdelta_status gdelta_set_wait_limit(uint32_t polls) {
+    g_wait_polls.store(polls == 0 ? kDefaultWaitPolls : polls, std::memory_order_relaxed);
+    return GDELTA_OK;
+}
+
+gdelta_status gdelta_set_wait_timeout_test(int32_t on) {
+    if (on != 0 && on != 1) return GDELTA_ERR_INVALID_ARG;
+    g_stall_test.store(on, std::memory_order_relaxed);
+    return GDELTA_OK;
 }
 
 gdelta_status gdelta_get_last_device_error(void *stream) {

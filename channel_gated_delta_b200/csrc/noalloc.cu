@@ -16,8 +16,9 @@
 namespace gdelta {
 
 // 32 MiB: the tensor-core forward needs 105 KiB per 64-token window of each
-// (batch, head), plus one int per window, so this holds 311 windows (for
-// example B = 1, H = 16, T <= 1216, or B * H = 8 with T <= 2432).
+// (batch, head), plus one int per window (the flags rounded up to 1 KiB), so
+// this holds 312 windows (for example B = 1, H = 16, T <= 1216, or B * H = 8
+// with T <= 2496).
 constexpr size_t kNoAllocScratchBytes = 32u << 20;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];

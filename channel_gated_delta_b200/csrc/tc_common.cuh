@@ -73,6 +73,20 @@ __device__ __forceinline__ uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn
     return d;
 }
 
+// Instruction descriptor, kind::f16 with bf16 A and B (format code 1 in both
+// operand fields), fp32 accumulator.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    uint32_t d = 0;
+    d |= 1u << 4;                              // D format: f32
+    d |= 1u << 7;                              // A format: bf16
+    d |= 1u << 10;                             // B format: bf16
+    d |= (a_mn ? 1u : 0u) << 15;
+    d |= (b_mn ? 1u : 0u) << 16;
+    d |= (uint32_t)(N >> 3) << 17;
+    d |= (uint32_t)(M >> 4) << 24;
+    return d;
+}
+
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                         uint32_t idesc, bool accumulate) {
     const uint32_t acc = accumulate ? 1u : 0u;
@@ -240,6 +254,18 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until all committed bulk stores are complete.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 2-D tiled TMA load of one box of the tensor map at `tmap` (a kernel parameter
+// in param space, passed by generic address) into this CTA's shared memory,
+// completion counted on the mbarrier.  x is the innermost coordinate (it must
+// be a multiple of 16 bytes' worth of elements); no multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst_smem),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
 
 // Hint: bring `bytes` (a multiple of 16) of global memory into L2.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {

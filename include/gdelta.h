@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GDELTA_ABI_VERSION 3
+#define GDELTA_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define GDELTA_API __attribute__((visibility("default")))
@@ -271,7 +271,7 @@ GDELTA_API gdelta_status gdelta_fwd_chunked(const gdelta_fwd_args *args, void *s
  *
  *  - Limit: gdelta_fwd_workspace_bytes(args) must not exceed 32 MiB (105 KiB
  *    per 64-token window of each batch row and head, plus one int per window:
- *    311 windows, e.g. B = 1, H = 16, T <= 1216).  Larger problems return
+ *    312 windows, e.g. B = 1, H = 16, T <= 1216, or B * H = 8, T <= 2496).  Larger problems return
  *    GDELTA_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up the array's device address (a CUDA
  *    runtime call); make that first call before capturing any stream.
@@ -286,6 +286,93 @@ GDELTA_API gdelta_status gdelta_fwd_chunked_noalloc(const gdelta_fwd_args *args,
 
 /* One decode step; see gdelta_decode_args. */
 GDELTA_API gdelta_status gdelta_decode_step(const gdelta_decode_args *args, void *stream);
+
+/*
+ * Five-gate low-rank projection: the fused prologue that produces the mixer's
+ * gates from the layer input (Muir review §2.3, "五门融合投影与参数再分配").
+ * The decay f, erase b, output g, write w and query-gain q gates share one
+ * down-projection of x whose width R is the sum of their ranks (the review's
+ * main model: 64, 64, 128, 128, 128; R = 512); each gate has its own
+ * up-projection back to d and a per-channel bias, which give its logits:
+ *
+ *   c        = x w_down                          [N, R]  (in the workspace)
+ *   logit_i  = c[:, R_i] w_up[R_i, :] + bias_i   [N, d]  R_i = gate i's block of R
+ *
+ * and the logits are activated into the form gdelta_fwd_chunked reads (the
+ * review fixes the ranges, not every activation; these are the plainest
+ * readings with those ranges):
+ *   log_alpha = log sigmoid(logit_f)  fp32 (alpha = sigmoid(logit_f) in (0, 1))
+ *   b = 2 sigmoid(logit_b)            bf16, in (0, 2)
+ *   g = sigmoid(logit_g), w = sigmoid(logit_w)   bf16, in (0, 1)
+ *   z = logit_q                       bf16 (the readout applies 2 sigmoid(z))
+ *
+ *   N          : tokens (rows), >= 1
+ *   d          : model width = H * d_head, a multiple of 256; the [N, d]
+ *                outputs are the mixer's [B, T, H, d_head] tensors when
+ *                N = B * T (heads contiguous, h-major)
+ *   ranks      : per gate in the order f, b, g, w, q; each a multiple of 64,
+ *                their sum R a multiple of 256 and at most 2048
+ *   x          : [N, d] bf16
+ *   w_down     : [d, R] bf16, columns grouped f | b | g | w | q
+ *   w_up       : [R, d] bf16, rows grouped the same way
+ *   bias       : [5, d] fp32, one row per gate in the same order
+ *   log_alpha  : [N, d] fp32 out;  b, g, w, z : [N, d] bf16 out
+ *   workspace  : gdelta_gate_proj_workspace_bytes(args) bytes of device memory
+ *                for the codes c (GDELTA_ERR_WORKSPACE if smaller)
+ * Both products run on tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation).  Between them the codes are held as two bf16 parts, c = hi +
+ * lo, and the up-projection reads both, so the codes keep about 16 bits (one
+ * bf16 part would shift the log-decay by several percent of its rms).  Asynchronous on
+ * `stream`; a bounded wait that runs out is reported by
+ * gdelta_get_last_device_error as GDELTA_ERR_TIMEOUT.
+ */
+typedef struct gdelta_gate_proj_args {
+    int32_t N, d;
+    int32_t ranks[5];
+    const void *x;
+    const void *w_down;
+    const void *w_up;
+    const float *bias;
+    float *log_alpha;
+    void *b, *g, *w, *z;
+    void *workspace;
+    size_t workspace_bytes;
+} gdelta_gate_proj_args;
+
+/* Workspace gdelta_gate_proj needs (0 if the arguments are invalid). */
+GDELTA_API size_t gdelta_gate_proj_workspace_bytes(const gdelta_gate_proj_args *args);
+
+/* Five-gate projection; see gdelta_gate_proj_args. */
+GDELTA_API gdelta_status gdelta_gate_proj(const gdelta_gate_proj_args *args, void *stream);
+
+/*
+ * Limit of the tensor-core kernels' bounded waits (failure detection; the
+ * papers specify no such limit).  Every wait of a tensor-core forward kernel on
+ * another party -- an MMA completion, a window record, the other CTA of its
+ * cluster, the readout warps -- polls its mbarrier at most `polls` times; when
+ * the limit runs out the kernel records GDELTA_ERR_TIMEOUT in the device status
+ * word, issues no further work, lets its own copies and MMAs in flight finish,
+ * frees its tensor memory and returns.  polls = 0 restores the default of
+ * 2^20 polls.  The setting is process-wide, read when a call is queued (calls
+ * already queued keep their limit), and applies to gdelta_fwd_chunked and
+ * gdelta_fwd_chunked_noalloc on the tensor-core path and to gdelta_gate_proj;
+ * the other kernels do not wait.  A limit far below the time the hardware needs turns ordinary waits
+ * into timeouts: the call then reports GDELTA_ERR_TIMEOUT and its outputs are
+ * unreliable, but the device stays usable.  Always returns GDELTA_OK.
+ */
+GDELTA_API gdelta_status gdelta_set_wait_limit(uint32_t polls);
+
+/*
+ * Failure-path test switch (no counterpart in the papers).  With on = 1 every
+ * call queued afterwards that gdelta_set_wait_limit governs first waits on an
+ * mbarrier that nothing ever completes, before it issues any copy or MMA; the
+ * wait runs out after the set limit, the kernels skip their work and return,
+ * and gdelta_get_last_device_error reports GDELTA_ERR_TIMEOUT.  The outputs of
+ * such a call are not written.  on = 0 (the default) turns it
+ * off.  Nothing faults or hangs: the failing wait is an ordinary bounded wait.
+ * Process-wide; returns GDELTA_ERR_INVALID_ARG for values other than 0 and 1.
+ */
+GDELTA_API gdelta_status gdelta_set_wait_timeout_test(int32_t on);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

@@ -44,6 +44,8 @@ __all__ = [
     "decode_step_inputs",
     "decode_gamma",
     "quantise",
+    "GATE_RANKS",
+    "gate_proj_inputs",
 ]
 
 TOKEN_KEYS = ("q", "k", "v", "b", "w", "z", "g")
@@ -203,3 +205,26 @@ def decode_step_inputs(step: int, seed: int = DECODE["seed"], B: int = DECODE["B
     out = _pack(raw, "bf16", np.ones((H, dk)))
     del out["gamma_stat"]
     return {key: val[:, 0] for key, val in out.items()}
+
+
+# Ranks of the five-gate projection in gate order f, b, g, w, q (the Muir
+# review's main model: 64, 64, 128, 128, 128; 512 in all).
+GATE_RANKS = (64, 64, 128, 128, 128)
+
+
+def gate_proj_inputs(N: int, d: int, ranks=GATE_RANKS, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Synthetic layer input and projection weights (no trained weights exist
+    here): x [N, d] ~ N(0, 1); w_down [d, R] ~ N(0, 1/d) so the codes have unit
+    variance; w_up [R, d] with each gate's rows ~ N(0, 1/r_gate) so every
+    logit has unit variance before its bias; all three in bf16.  Biases [5, d]
+    fp32: the decay gate's ~ U(2, 7), the decay logits of the workloads'
+    log-decays -exp(u), u ~ U(-7, -2); the other gates' 0."""
+    R = int(sum(ranks))
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 7])))
+    x = rng.standard_normal((N, d))
+    w_down = rng.standard_normal((d, R)) / np.sqrt(d)
+    w_up = np.concatenate([rng.standard_normal((r, d)) / np.sqrt(r) for r in ranks])
+    bias = np.zeros((len(ranks), d))
+    bias[0] = rng.uniform(2.0, 7.0, d)
+    return {"x": quantise(x, "bf16"), "w_down": quantise(w_down, "bf16"), "w_up": quantise(w_up, "bf16"),
+            "bias": torch.from_numpy(bias).to(torch.float32)}

@@ -16,6 +16,7 @@ struct SelftestParams {
     int a_mn, b_mn, a_neg;
     int RA, a_row0, RB, b_row0;
     int *err;
+    int d_lane;          // M = 64 only: lane offset of the accumulator (0 or 16)
 };
 
 __global__ void __launch_bounds__(128) tc_selftest_kernel(SelftestParams p) {
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(128) tc_selftest_kernel(SelftestParams p) {
         for (int ks = 0; ks < p.K / 16; ++ks) {
             const uint64_t ad = p.a_mn ? desc_mnmajor(a0, p.RA, p.a_row0, ks) : desc_kmajor(a0, p.RA, p.a_row0, ks);
             const uint64_t bd = p.b_mn ? desc_mnmajor(b0, p.RB, p.b_row0, ks) : desc_kmajor(b0, p.RB, p.b_row0, ks);
-            mma_f16(taddr, ad, bd, id, ks > 0);
+            mma_f16(taddr + ((uint32_t)p.d_lane << 16), ad, bd, id, ks > 0);
         }
         mma_commit(smem_u32(mbar));
     }
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(128) tc_selftest_kernel(SelftestParams p) {
             tmem_ld32(taddr + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
             int row = -1;
             if (p.M == 128) row = 32 * warp + lane;
-            else if (lane < 16) row = 16 * warp + lane;
+            else if (lane >= p.d_lane && lane < p.d_lane + 16) row = 16 * warp + lane - p.d_lane;
             if (row >= 0)
                 for (int i = 0; i < 32 && c + i < p.N; ++i) p.D[row * p.N + c + i] = v[i];
         }
@@ -83,8 +84,9 @@ __global__ void __launch_bounds__(128) tc_selftest_kernel(SelftestParams p) {
 }
 
 extern "C" int tc_selftest(const float *A, const float *B, float *D, int M, int N, int K, int a_mn, int b_mn,
-                           int a_neg, int RA, int a_row0, int RB, int b_row0, int *err, void *stream) {
-    SelftestParams p{A, B, D, M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0, err};
+                           int a_neg, int RA, int a_row0, int RB, int b_row0, int d_lane, int *err, void *stream) {
+    SelftestParams p{A, B, D, M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0, err, d_lane};
+    if (d_lane != 0 && !(M == 64 && d_lane == 16)) return 2;
     const int colsA = a_mn ? M : K, colsB = b_mn ? N : K;
     // bounds of every access, checked on the host before the launch
     if ((M != 64 && M != 128) || N % 32 || N < 32 || N > 256 || K % 16 || K < 16) return 2;

@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.gdelta_abi_version() == 3
+    assert lib.gdelta_abi_version() == 4
     for code in range(8):
         s = lib.gdelta_status_string(code)
         assert s and s != b"unknown status"

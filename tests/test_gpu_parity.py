@@ -108,7 +108,7 @@ def test_split_run_carries_state():
 @pytest.mark.parametrize("name,heads", [
     ("layer350m_bf16", [(0, 0), (3, 5), (7, 7)]),
     ("muir1b3_bf16", [(0, 0), (1, 9), (3, 15)]),
-    ("long32k_bf16", [(0, 0), (0, 11)]),
+    ("long32k_bf16", [(0, 0), (0, 11), (0, 15)]),
 ])
 def test_full_size_configs_sampled_heads(name, heads):
     """Full workload in the benchmark's launch configuration; the oracle

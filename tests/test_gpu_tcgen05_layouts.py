@@ -31,11 +31,11 @@ def build_selftest():
 def lib():
     l = ctypes.CDLL(build_selftest())
     l.tc_selftest.restype = ctypes.c_int
-    l.tc_selftest.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 10 + [ctypes.c_void_p] * 2
+    l.tc_selftest.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 11 + [ctypes.c_void_p] * 2
     return l
 
 
-# (M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0, what)
+# (M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0, what[, d_lane])
 CASES = [
     (128, 128, 128, 0, 0, 0, 128, 0, 128, 0, "decay products: K-major A and B"),
     (64, 128, 64, 0, 1, 0, 64, 0, 128, 0, "W' = Tinv Kp: MN-major B from the top half of a 128-row tile"),
@@ -47,12 +47,14 @@ CASES = [
     (128, 64, 128, 0, 1, 0, 128, 0, 128, 0, "[W';Q] S_c, one value half"),
     (128, 256, 64, 0, 0, 0, 128, 0, 256, 0, "N = 256, K-major B"),
     (64, 192, 64, 0, 1, 0, 64, 0, 64, 0, "N = 192, MN-major B with three column blocks"),
+    (64, 64, 64, 0, 1, 0, 64, 0, 64, 0, "M = 64 accumulator in the upper half of each lane quadrant", 16),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=[c[-1] for c in CASES])
+@pytest.mark.parametrize("case", CASES, ids=[c[10] for c in CASES])
 def test_tcgen05_operand_view(lib, case):
-    M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0, _ = case
+    M, N, K, a_mn, b_mn, a_neg, RA, a_row0, RB, b_row0 = case[:10]
+    d_lane = case[11] if len(case) > 11 else 0
     g = torch.Generator().manual_seed(M * 7 + N + K + a_row0)
     A = torch.randn(M, K, generator=g)
     B = torch.randn(K, N, generator=g)
@@ -61,7 +63,7 @@ def test_tcgen05_operand_view(lib, case):
     dD = torch.full((M, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = lib.tc_selftest(dA.data_ptr(), dB.data_ptr(), dD.data_ptr(), M, N, K, a_mn, b_mn, a_neg, RA, a_row0,
-                         RB, b_row0, err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                         RB, b_row0, d_lane, err.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert rc == 0
     torch.cuda.synchronize()
     assert int(err.item()) == 0, "mbarrier wait ran out"

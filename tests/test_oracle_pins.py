@@ -313,6 +313,51 @@ def test_rmsnorm_mean_of_squares():
         assert np.max(np.abs(ms_y - ms_o / (ms_o + eps))) < 1e-13
 
 
+def test_readout_gain_limits_of_the_dynamic_modulation():
+    """The dynamic readout modulation 2 sigmoid(z) spans (0, 2) (Muir review
+    §2.1): z -> +inf doubles the z = 0 readout, z -> -inf silences it, and the
+    state never sees z."""
+    T, dk, dv = 9, 8, 6
+    d = rand_inputs(T, dk, dv, seed=41)
+    base = oracle.forward(dict(d, z=np.zeros_like(d["z"])))
+    hi = oracle.forward(dict(d, z=np.full_like(d["z"], 40.0)))
+    lo = oracle.forward(dict(d, z=np.full_like(d["z"], -40.0)))
+    scale = np.max(np.abs(base["o_raw"]))
+    assert np.max(np.abs(hi["o_raw"] - 2.0 * base["o_raw"])) <= 1e-14 * scale
+    assert np.max(np.abs(lo["o_raw"])) <= 1e-15 * scale
+    assert np.max(np.abs(lo["y"])) <= 1e-6          # g * 0 / sqrt(0 + eps)
+    for r in (hi, lo, oracle.forward(d)):
+        assert np.array_equal(r["S"], base["S"])
+
+
+def test_static_gain_scales_query_channels_and_never_the_state():
+    """gamma_stat multiplies the query channel-wise (Muir review §2.1, a
+    query-only gain): with a one-hot profile e_i and z = 0 the readout of
+    token t is q_ti times row i of the state after token t (read after write),
+    the state is the same for every profile, and a uniform profile c scales
+    o_raw by c and leaves y as it is (RMSNorm, exactly when eps = 0)."""
+    T, dk, dv, i = 6, 8, 5, 3
+    d = rand_inputs(T, dk, dv, seed=43)
+    d["z"] = np.zeros_like(d["z"])
+    one_hot = np.zeros_like(d["gamma_stat"])
+    one_hot[0, i] = 1.0
+    r = oracle.forward(dict(d, gamma_stat=one_hot))
+    for t in range(T):
+        prefix = {k: (v[:, :t + 1] if v.ndim == 4 else v) for k, v in d.items()}
+        S_t = oracle.forward(prefix)["S"][0]                 # state after token t
+        want = d["q"][0, t, 0, i] * S_t[i]
+        assert np.max(np.abs(r["o_raw"][0, t] - want)) <= 1e-13 * max(np.max(np.abs(S_t)), 1e-300)
+    base = oracle.forward(d)
+    assert np.array_equal(r["S"], base["S"])
+    c = 3.5
+    scaled = oracle.forward(dict(d, gamma_stat=c * d["gamma_stat"]))
+    assert np.array_equal(scaled["S"], base["S"])
+    assert relerr(scaled["o_raw"], c * base["o_raw"]) <= 1e-14
+    # with eps = 0 RMSNorm removes the scale exactly
+    y0, y0c = oracle.forward(d, eps=0.0)["y"], oracle.forward(dict(d, gamma_stat=c * d["gamma_stat"]), eps=0.0)["y"]
+    assert relerr(y0c, y0) <= 1e-13
+
+
 def test_golden_readback_squared_norm():
     """A single association S = k^T v read with the same unnormalised key
     returns |k|^2 v ("Kimi3 = GPT2 x 22580" §3)."""
