@@ -19,8 +19,9 @@
 // A CTA runs one SM: warp 0 stages A and B tiles with TMA into a 4-deep ring
 // (128-byte swizzle, the layout the MMA descriptors read), warp 1 issues the
 // MMAs (M = 128 tokens, N = 256 columns, K = 64 per stage) into one of two
-// TMEM accumulators, warps 2-5 drain the other accumulator (bias, activation,
-// stores) meanwhile.
+// TMEM accumulators, warps 2-9 drain the other accumulator (bias, activation,
+// stores) meanwhile: two warps per 32-lane TMEM quadrant, one per half of the
+// tile's columns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -38,7 +39,8 @@ constexpr int kPStages = 4;
 constexpr int kPATile = kPM * kPK * 2;            // 16 KiB
 constexpr int kPBTile = kPK * kPN * 2;            // 32 KiB: 4 column blocks of 64 x 64
 constexpr int kPStage = kPATile + kPBTile;
-constexpr int kPThreads = 192;
+constexpr int kPThreads = 320;                   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kPEpiWarps = 8;
 constexpr uint32_t kPDrainPolls = 1u << 22;
 
 struct ProjSmem {
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(s_accf + 8 * b, 1);
-            tc::mbar_init(s_acce + 8 * b, 4);
+            tc::mbar_init(s_acce + 8 * b, kPEpiWarps);
         }
         tc::mbar_init(s_stall, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -216,8 +218,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
             }
         }
     } else if (warp >= 2) {
-        // ---- epilogue: TMEM lanes 32 (warp % 4) .. +31 are the tile's rows
-        const int qd = warp & 3, row = 32 * qd + lane;
+        // ---- epilogue: TMEM lanes 32 (warp % 4) .. +31 are the tile's rows; warps
+        // 2-5 take columns 0-127 of the tile, warps 6-9 columns 128-255
+        const int qd = warp & 3, row = 32 * qd + lane, cbase = warp < 6 ? 0 : kPN / 2;
         uint32_t t = 0;
         for (int j = blockIdx.x; j < p.jobs; j += gridDim.x, ++t) {
             const Job jb = job_of(p, j);
@@ -233,10 +236,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const uint32_t acc = tmem + ((uint32_t)(32 * qd) << 16) + b * kPN;
             const int m = jb.m0 + row;
             const bool live = m < p.M;
-            for (int c = 0; c < kPN / 32; ++c) {
+            for (int c = 0; c < kPN / 64; ++c) {
                 float x[32];
-                tc::tmem_ld32(acc + 32 * c, x);
-                const int n = jb.n0 + 32 * c;
+                tc::tmem_ld32(acc + cbase + 32 * c, x);
+                const int n = jb.n0 + cbase + 32 * c;
                 if (!p.up) {
                     if (live) {
                         // c = hi + lo: hi its bf16 rounding, lo the bf16 rounding of the rest
