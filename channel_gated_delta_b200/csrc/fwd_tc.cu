@@ -460,57 +460,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     float *lw = (float *)(xbuf + L::LW), *yb = (float *)(xbuf + L::YB);
                     const uint32_t s_ti = tc::smem_u32(xbuf + L::TI), s_mm = tc::smem_u32(xbuf + L::MM);
                     const int tb = 8 * warp, c4 = 4 * lane;
-                    float la[8][4];
-                    uint2 kq[8][4];                           // [token][k, q, z, b]: 4 bf16 each
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int t = tb + u;
-                        const bool in = t0 + t < wend;
-                        const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gk = gt * kDK + c4;
+                    // token u's inputs, loaded one token ahead of their use below so that a
+                    // thread never holds more than two tokens' worth (a register peak here
+                    // would make the whole chain kernel spill)
+                    auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
+                    auto load_la = [&](int u) -> float4 {
                         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (in) {
+                        if (t0 + tb + u < wend) {
                             if (p.decay_tok) {
-                                const float s = __ldg(p.la + gt);
-                                x = make_float4(s, s, s, s);
+                                const float sc = __ldg(p.la + gt_of(u));
+                                x = make_float4(sc, sc, sc, sc);
                             } else {
-                                x = __ldg(reinterpret_cast<const float4 *>(p.la + gk));
+                                x = __ldg(reinterpret_cast<const float4 *>(p.la + gt_of(u) * kDK + c4));
                             }
                         }
-                        la[u][0] = x.x; la[u][1] = x.y; la[u][2] = x.z; la[u][3] = x.w;
-                        kq[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
-                        kq[u][1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-                        kq[u][2] = in && p.z ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-                        kq[u][3] = !in ? make_uint2(0, 0)
-                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
-                    }
-                    // inclusive scan over tokens: within this warp's 8 tokens, then across warps
-#pragma unroll
-                    for (int u = 1; u < 8; ++u)
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) la[u][c] += la[u - 1][c];
-                    *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(la[7][0], la[7][1], la[7][2], la[7][3]);
-                    main_sync();
+                        return x;
+                    };
+                    auto load_kq = [&](int u, uint2 (&o)[4]) {        // k, q, z, b: 4 bf16 each
+                        const bool in = t0 + tb + u < wend;
+                        const size_t gt = gt_of(u), gk = gt * kDK + c4;
+                        o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
+                        o[1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
+                        o[2] = in && p.z ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+                        o[3] = !in ? make_uint2(0, 0)
+                              : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
+                    };
+                    auto load_vw = [&](int u, uint2 (&o)[2]) {        // v, w of this CTA's value columns
+                        const bool in = t0 + tb + u < wend && c4 < kDVC;
+                        const size_t gt = gt_of(u), gv = gt * kDV + dv0 + c4;
+                        o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+                        o[1] = !in ? make_uint2(0, 0)
+                              : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                    };
+                    // inclusive scan over tokens: this warp's sum (and its prefix at tokens
+                    // 0, 1, 3 and 7 of the warp, the probe tokens it may own), then across warps
+                    float off[4] = {0.f, 0.f, 0.f, 0.f};
                     {
-                        float off[4] = {0.f, 0.f, 0.f, 0.f};
+                        float run[4] = {0.f, 0.f, 0.f, 0.f}, pre[4][4];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float4 x = load_la(u);
+                            run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
+                            const int j = u == 0 ? 0 : u == 1 ? 1 : u == 3 ? 2 : u == 7 ? 3 : -1;
+                            if (j >= 0)
+#pragma unroll
+                                for (int c = 0; c < 4; ++c) pre[j][c] = run[c];
+                        }
+                        *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(run[0], run[1], run[2], run[3]);
+                        main_sync();
                         for (int ww = 0; ww < warp; ++ww) {
                             const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
                             off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
                         }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) la[u][c] += off[c];        // la now holds Lambda_t
-                    }
-                    // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j)
-#pragma unroll
-                    for (int j = 0; j < 7; ++j) {
-                        const int pt = (1 << j) - 1;
-                        if (pt >= tb && pt < tb + 8) {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                if (tb + u == pt)
-                                    *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
-                                        make_float4(la[u][0], la[u][1], la[u][2], la[u][3]);
+                        // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j):
+                        // tokens 0-7 are warp 0's, 15 warp 1's, 31 warp 3's, 63 warp 7's last
+                        auto put = [&](int j, int k) {
+                            *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
+                                make_float4(off[0] + pre[k][0], off[1] + pre[k][1], off[2] + pre[k][2], off[3] + pre[k][3]);
+                        };
+                        if (warp == 0) {
+                            put(0, 0);
+                            put(1, 1);
+                            put(2, 2);
+                            put(3, 3);
+                        } else if (warp == 1) {
+                            put(4, 3);
+                        } else if (warp == 3) {
+                            put(5, 3);
+                        } else if (warp == 7) {
+                            put(6, 3);
                         }
                     }
                     main_sync();
@@ -541,18 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         flags[1] = min(1 << nj, wend - t0);
                         flags[2] = nj;
                     }
-                    // value-side loads (their latency overlaps the operand computation)
                     const bool vlane = c4 < kDVC;
-                    uint2 vw[8][2];                           // [token][v, w]
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int t = tb + u;
-                        const bool in = t0 + t < wend && vlane;
-                        const size_t gt = ((size_t)bb * T + t0 + t) * H + h, gv = gt * kDV + dv0 + c4;
-                        vw[u][0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                        vw[u][1] = !in ? make_uint2(0, 0)
-                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
-                    }
                     main_sync();
                     n = flags[1];
 
@@ -576,16 +583,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                                 fcv[c4 + c] = __expf(lnv[c] - cpiv[c]);
                             }
                         }
+                        float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
+                        float4 la_nx = load_la(0);
+                        uint2 kq_nx[4];
+                        load_kq(0, kq_nx);
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
                             const int t = tb + u;
                             const bool live = t < n;
+                            const float4 la_c = la_nx;
+                            const uint2 kq_c[4] = {kq_nx[0], kq_nx[1], kq_nx[2], kq_nx[3]};
+                            if (u + 1 < 8) {
+                                la_nx = load_la(u + 1);
+                                load_kq(u + 1, kq_nx);
+                            }
+                            lam_run[0] += la_c.x; lam_run[1] += la_c.y; lam_run[2] += la_c.z; lam_run[3] += la_c.w;
                             float kk[4], qq[4], zz[4], bv[4];
                             {
-                                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][0]);
-                                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][1]);
-                                const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][2]);
-                                const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq[u][3]);
+                                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[0]);
+                                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[1]);
+                                const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[2]);
+                                const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[3]);
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     float2 f;
@@ -603,7 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                             float dq = 0.f, db = 0.f;
 #pragma unroll
                             for (int c = 0; c < 4; ++c) {
-                                const float lam = live ? la[u][c] : lnv[c];     // identity padding past n
+                                const float lam = live ? lam_run[c] : lnv[c];   // identity padding past n
                                 const float d = lam - cpiv[c];
                                 const float ep = __expf(d), em = __expf(-d);
                                 const float kv = live ? kk[c] : 0.f;
@@ -638,12 +656,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                                 make_uint2(tc::pack_half2(khc[0], khc[1]), tc::pack_half2(khc[2], khc[3]));
                         }
                         if (vlane) {
+                            uint2 vw_nx[2];
+                            load_vw(0, vw_nx);
 #pragma unroll
                             for (int u = 0; u < 8; ++u) {
                                 const int t = tb + u;
                                 const bool live = t < n;
-                                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][0]);
-                                const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw[u][1]);
+                                const uint2 vw_c[2] = {vw_nx[0], vw_nx[1]};
+                                if (u + 1 < 8) load_vw(u + 1, vw_nx);
+                                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
+                                const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
                                 float vh[4];
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
