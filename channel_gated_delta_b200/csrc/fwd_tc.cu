@@ -446,372 +446,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 inflight[B ^ 1] = false;
             }
             main_sync();
-            for (int t0 = kC * w; t0 < wend && flags[0] == 0;) {
-                int n = wend - t0;
+            // The products of one chunk (H to K) on the tiles in `buf`.  Called from two
+            // places: a precomputed window is one chunk and takes the first call alone,
+            // so its code stays compact; windows processed in shorter chunks build the
+            // tiles first (a large block that, placed in line before the products,
+            // measured 3 % slower on windows that never use it).
+            auto chunk_products = [&](const int t0, const int n) {
                 const uint32_t slot = (uint32_t)(chunk & 1);      // TMEM slot of this chunk's [R; O]
                 const uint32_t ro = kTmRO + (uint32_t)kDVC * slot;
                 ++chunk;
-                if (!fast && flags[0] == 0) do {
-                    // ---- A: loads, cumulative log-decay, span, chunk length.
-                    // Warp w owns tokens [8w, 8w+8); lane l owns key channels [4l, 4l+4)
-                    // and, for l < 16, value channels dv0 + [4l, 4l+4).
-                    float *wtot = (float *)(xbuf + L::WT), *probe = (float *)(xbuf + L::PR);
-                    float *spanred = (float *)(xbuf + L::XV), *diagq = spanred + 64, *diagb = spanred + 128;
-                    float *lw = (float *)(xbuf + L::LW), *yb = (float *)(xbuf + L::YB);
-                    const uint32_t s_ti = tc::smem_u32(xbuf + L::TI), s_mm = tc::smem_u32(xbuf + L::MM);
-                    const int tb = 8 * warp, c4 = 4 * lane;
-                    // token u's inputs, loaded one token ahead of their use below so that a
-                    // thread never holds more than two tokens' worth (a register peak here
-                    // would make the whole chain kernel spill)
-                    auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
-                    auto load_la = [&](int u) -> float4 {
-                        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (t0 + tb + u < wend) {
-                            if (p.decay_tok) {
-                                const float sc = __ldg(p.la + gt_of(u));
-                                x = make_float4(sc, sc, sc, sc);
-                            } else {
-                                x = __ldg(reinterpret_cast<const float4 *>(p.la + gt_of(u) * kDK + c4));
-                            }
-                        }
-                        return x;
-                    };
-                    auto load_kq = [&](int u, uint2 (&o)[4]) {        // k, q, z, b: 4 bf16 each
-                        const bool in = t0 + tb + u < wend;
-                        const size_t gt = gt_of(u), gk = gt * kDK + c4;
-                        o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
-                        o[1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-                        o[2] = in && p.z ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-                        o[3] = !in ? make_uint2(0, 0)
-                              : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
-                    };
-                    auto load_vw = [&](int u, uint2 (&o)[2]) {        // v, w of this CTA's value columns
-                        const bool in = t0 + tb + u < wend && c4 < kDVC;
-                        const size_t gt = gt_of(u), gv = gt * kDV + dv0 + c4;
-                        o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                        o[1] = !in ? make_uint2(0, 0)
-                              : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
-                    };
-                    // inclusive scan over tokens: this warp's sum (and its prefix at tokens
-                    // 0, 1, 3 and 7 of the warp, the probe tokens it may own), then across warps
-                    float off[4] = {0.f, 0.f, 0.f, 0.f};
-                    {
-                        float run[4] = {0.f, 0.f, 0.f, 0.f}, pre[4][4];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float4 x = load_la(u);
-                            run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
-                            const int j = u == 0 ? 0 : u == 1 ? 1 : u == 3 ? 2 : u == 7 ? 3 : -1;
-                            if (j >= 0)
-#pragma unroll
-                                for (int c = 0; c < 4; ++c) pre[j][c] = run[c];
-                        }
-                        *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(run[0], run[1], run[2], run[3]);
-                        main_sync();
-                        for (int ww = 0; ww < warp; ++ww) {
-                            const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
-                            off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
-                        }
-                        // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j):
-                        // tokens 0-7 are warp 0's, 15 warp 1's, 31 warp 3's, 63 warp 7's last
-                        auto put = [&](int j, int k) {
-                            *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
-                                make_float4(off[0] + pre[k][0], off[1] + pre[k][1], off[2] + pre[k][2], off[3] + pre[k][3]);
-                        };
-                        if (warp == 0) {
-                            put(0, 0);
-                            put(1, 1);
-                            put(2, 2);
-                            put(3, 3);
-                        } else if (warp == 1) {
-                            put(4, 3);
-                        } else if (warp == 3) {
-                            put(5, 3);
-                        } else if (warp == 7) {
-                            put(6, 3);
-                        }
-                    }
-                    main_sync();
-                    {
-                        // span of a chunk of 2^j tokens: max over this thread's 4 channels, then the CTA
-                        const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
-                        float sp[7];
-#pragma unroll
-                        for (int j = 0; j < 7; ++j) {
-                            const float4 lj = *reinterpret_cast<const float4 *>(probe + j * kDK + c4);
-                            float m = fmaxf(fmaxf(l0.x - lj.x, l0.y - lj.y), fmaxf(l0.z - lj.z, l0.w - lj.w));
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                            sp[j] = m;
-                        }
-                        if (lane == 0)
-#pragma unroll
-                            for (int j = 0; j < 7; ++j) spanred[warp * 8 + j] = sp[j];
-                    }
-                    main_sync();
-                    if (tid == 0) {
-                        int nj = 0;
-                        for (int j = 6; j >= 0; --j) {
-                            float m = 0.f;
-                            for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, spanred[ww * 8 + j]);
-                            if (m <= kSpanMax) { nj = j; break; }
-                        }
-                        flags[1] = min(1 << nj, wend - t0);
-                        flags[2] = nj;
-                    }
-                    const bool vlane = c4 < kDVC;
-                    main_sync();
-                    n = flags[1];
-
-                    // ---- B: operand tiles (fp16, swizzled), pivot vectors, exact diagonals
-                    {
-                        // Lambda_{n-1} is the probe of the chosen power-of-two chunk: past the
-                        // end of the sequence the log-decay is zero-padded, so a shorter tail
-                        // has the same cumulative value there.
-                        const int jn = flags[2];
-                        const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
-                        const float4 ln4 = *reinterpret_cast<const float4 *>(probe + jn * kDK + c4);
-                        const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
-                        const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
-                        float cpiv[4], gq[4];
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            cpiv[c] = 0.5f * (l0v[c] + lnv[c]);
-                            gq[c] = gsv[c4 + c];
-                            if (warp == 0) {
-                                ecv[c4 + c] = __expf(cpiv[c]);
-                                fcv[c4 + c] = __expf(lnv[c] - cpiv[c]);
-                            }
-                        }
-                        float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
-                        float4 la_nx = load_la(0);
-                        uint2 kq_nx[4];
-                        load_kq(0, kq_nx);
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int t = tb + u;
-                            const bool live = t < n;
-                            const float4 la_c = la_nx;
-                            const uint2 kq_c[4] = {kq_nx[0], kq_nx[1], kq_nx[2], kq_nx[3]};
-                            if (u + 1 < 8) {
-                                la_nx = load_la(u + 1);
-                                load_kq(u + 1, kq_nx);
-                            }
-                            lam_run[0] += la_c.x; lam_run[1] += la_c.y; lam_run[2] += la_c.z; lam_run[3] += la_c.w;
-                            float kk[4], qq[4], zz[4], bv[4];
-                            {
-                                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[0]);
-                                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[1]);
-                                const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[2]);
-                                const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[3]);
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    float2 f;
-                                    f = __bfloat1622float2(hk[e]); kk[2 * e] = f.x; kk[2 * e + 1] = f.y;
-                                    f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
-                                    f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
-                                    f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
-                                }
-                                if (kRaw) {                 // the q/k preprocessing, one token a call
-                                    silu_l2n_row4(kk);
-                                    silu_l2n_row4(qq);
-                                }
-                            }
-                            float kp[4], kc[4], khc[4], qp[4];
-                            float dq = 0.f, db = 0.f;
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const float lam = live ? lam_run[c] : lnv[c];   // identity padding past n
-                                const float d = lam - cpiv[c];
-                                const float ep = __expf(d), em = __expf(-d);
-                                const float kv = live ? kk[c] : 0.f;
-                                const float qt = live ? qq[c] * gq[c] * (2.f / (1.f + __expf(-zz[c]))) : 0.f;
-                                const float kh = bv[c] * kv;
-                                dq += qt * kv;
-                                db += qt * kh;
-                                kp[c] = kv * ep;
-                                kc[c] = kv * em;
-                                khc[c] = kh * em;
-                                qp[c] = qt * ep;
-                            }
-                            range_max = fmaxf(range_max, fmaxf(fmaxf(maxabs(kp, 4), maxabs(kc, 4)),
-                                                               fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
-                            // the diagonal of Aq / Bq carries no decay: it is summed exactly in
-                            // fp32 (a readout whose q~.k nearly cancels, e.g. the first token of a
-                            // sequence, is then free of fp16 operand rounding)
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) {
-                                dq += __shfl_xor_sync(0xffffffffu, dq, o);
-                                db += __shfl_xor_sync(0xffffffffu, db, o);
-                            }
-                            if (lane == 0) {
-                                diagq[t] = dq;
-                                diagb[t] = db;
-                            }
-                            const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
-                            *(uint2 *)(buf + L::AP + off_t) = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
-                            *(uint2 *)(buf + L::AP + off_b) = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
-                            *(uint2 *)(buf + L::BP + off_t) = make_uint2(tc::pack_half2(kc[0], kc[1]), tc::pack_half2(kc[2], kc[3]));
-                            *(uint2 *)(buf + L::BP + off_b) =
-                                make_uint2(tc::pack_half2(khc[0], khc[1]), tc::pack_half2(khc[2], khc[3]));
-                        }
-                        if (vlane) {
-                            uint2 vw_nx[2];
-                            load_vw(0, vw_nx);
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int t = tb + u;
-                                const bool live = t < n;
-                                const uint2 vw_c[2] = {vw_nx[0], vw_nx[1]};
-                                if (u + 1 < 8) load_vw(u + 1, vw_nx);
-                                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
-                                const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
-                                float vh[4];
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const float2 fv = __bfloat1622float2(hv[e]), fw = __bfloat1622float2(hw[e]);
-                                    vh[2 * e] = live ? fv.x * fw.x : 0.f;
-                                    vh[2 * e + 1] = live ? fv.y * fw.y : 0.f;
-                                }
-                                *(uint2 *)(buf + L::VH + tc::tile_off(64, t, c4)) =
-                                    make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
-                            }
-                        }
-                    }
-                    tc::fence_proxy_async();
-                    main_sync();
-
-                    // ---- C: decay-relative products P = [Kp; Qp] [Kc; K^c]^T
-                    if (tid == 0) {
-                        tc::fence_after_sync();
-                        const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
-                        for (int ks = 0; ks < kDK / 16; ++ks)
-                            tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id,
-                                        ks > 0);
-                        tc::mma_commit(s_mbar);
-                    }
-                    if (!wait_mma()) break;
-
-                    // ---- D: masks; M -> MM, L -> fp32, Aq/Bq -> ANAB
-                    {
-                        // rows 0-63: warps 0,1 (M, cols 0-63) and warps 4,5 (L, cols 64-127)
-                        // rows 64-127: warps 2,3 (Aq) and warps 6,7 (Bq)
-                        const int t = row & 63;
-                        const bool upper = row < 64;
-                        float v[2][32];
-                        tc::tmem_ld32x2(tmem + lane_base + kTmP + 64 * colhalf, tmem + lane_base + kTmP + 64 * colhalf + 32,
-                                        v[0], v[1]);
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const int s = 32 * hf + i;
-                                const bool keep = upper ? (s < t) : (s <= t);
-                                if (!keep) v[hf][i] = 0.f;
-                                if (!upper && s == t) v[hf][i] = colhalf == 0 ? diagq[t] : diagb[t];
-                            }
-                            if (upper && colhalf == 1) {
-                                float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    dst[q] = make_float4(v[hf][4 * q], v[hf][4 * q + 1], v[hf][4 * q + 2], v[hf][4 * q + 3]);
-                            } else {
-                                uint8_t *tile = upper ? xbuf + L::MM : buf + L::ANAB;
-                                const int R = upper ? 64 : 192;
-                                const int r = upper ? t : (colhalf == 0 ? 64 + t : 128 + t);
-                                store_row32(tile, R, r, 32 * hf, v[hf]);
-                            }
-                        }
-                    }
-                    tc::fence_before_sync();
-                    main_sync();
-
-                    // ---- E: T^-1 = (I + L)^-1 in place, divide and conquer (fp32)
-                    {
-                        // leaves of 8: forward substitution per column, in registers
-                        if (tid < 64) {
-                            const int o = 8 * (tid >> 3), j = tid & 7;
-                            float Lr[8][8];
-#pragma unroll
-                            for (int i = 1; i < 8; ++i)
-#pragma unroll
-                                for (int s = 0; s < i; ++s) Lr[i][s] = lw[(o + i) * kLW + o + s];
-                            float x[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) x[i] = (i == j) ? 1.f : 0.f;
-#pragma unroll
-                            for (int i = 1; i < 8; ++i) {
-                                float acc = 0.f;
-#pragma unroll
-                                for (int s = 0; s < i; ++s) acc += Lr[i][s] * x[s];
-                                if (i > j) x[i] = -acc;
-                            }
-                            __syncwarp();
-                            asm volatile("bar.sync 2, 64;" ::: "memory");     // the 64 leaf threads only
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                if (i >= j) lw[(o + i) * kLW + o + j] = x[i];
-                        }
-                        main_sync();
-                        // merges: [[A, 0], [C, D]]^-1 = [[A^-1, 0], [-D^-1 C A^-1, D^-1]],
-                        // four output columns per task; the upper triangles are zero, so the
-                        // sums run over whole blocks without masks
-                        merge_level<8>(lw, yb, tid);
-                        merge_level<16>(lw, yb, tid);
-                        merge_level<32>(lw, yb, tid);
-                        // T^-1 -> fp16 tile (row t, column s; the upper part of lw is zero)
-                        for (int u = tid; u < 64 * 8; u += kThreads) {
-                            const int t = u >> 3, g8 = u & 7;
-                            const float4 a = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8);
-                            const float4 b4 = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8 + 4);
-                            const float f[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-                            *(uint4 *)(xbuf + L::TI + tc::tile_chunk_off(64, t, g8)) = pack8(f);
-                        }
-                    }
-                    tc::fence_proxy_async();
-                    main_sync();
-
-                    // ---- F: W' = T^-1 Kp, N = T^-1 M
-                    if (tid == 0) {
-                        tc::fence_after_sync();
-                        const uint32_t idw = tc::idesc_f16(64, 128, false, true, false);
-                        const uint32_t idn = tc::idesc_f16(64, 64, false, true, false);
-                        for (int ks = 0; ks < kC / 16; ++ks)
-                            tc::mma_f16(tmem + kTmW, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_ap, 128, 0, ks), idw,
-                                        ks > 0);
-                        for (int ks = 0; ks < kC / 16; ++ks)
-                            tc::mma_f16(tmem + kTmN, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_mm, 64, 0, ks), idn,
-                                        ks > 0);
-                        tc::mma_commit(s_mbar);
-                    }
-                    if (!wait_mma()) break;
-
-                    // ---- G: W' -> rows 0-63 of AP (over Kp), N -> rows 0-63 of ANAB.
-                    // M = 64 accumulators sit in lanes 0-15 of each 32-lane group.
-                    {
-                        const int t = 16 * (warp & 3) + lane;
-                        const bool valid = lane < 16;
-                        float v[2][32];
-                        // warps 0-3: W' columns 0-63; warps 4-7: W' columns 64-127
-                        tc::tmem_ld32x2(tmem + lane_base + kTmW + 64 * colhalf, tmem + lane_base + kTmW + 64 * colhalf + 32,
-                                        v[0], v[1]);
-                        if (valid) {
-#pragma unroll
-                            for (int hf = 0; hf < 2; ++hf) {
-                                range_max = fmaxf(range_max, maxabs(v[hf], 32));
-                                store_row32(buf + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
-                            }
-                        }
-                        // warps 0-3: N columns 0-31; warps 4-7: N columns 32-63
-                        float nv[32];
-                        tc::tmem_ld32(tmem + lane_base + kTmN + 32 * colhalf, nv);
-                        if (valid) {
-                            range_max = fmaxf(range_max, maxabs(nv, 32));
-                            store_row32(buf + L::ANAB, 192, t, 32 * colhalf, nv);
-                        }
-                    }
-                } while (false);
-
                 if (flags[0] == 0) {
                     // ---- H: state operand S_c = Diag(e^c) S, X <- S_c (fp32, TMEM)
                     {
@@ -923,7 +566,375 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 main_sync();
                 tc::fence_after_sync();
                 ++uses[slot];
-                t0 += n;
+            };
+            if (fast) {
+                if (flags[0] == 0) chunk_products(kC * w, wend - kC * w);
+            } else {
+                for (int t0 = kC * w; t0 < wend && flags[0] == 0;) {
+                    int n = wend - t0;
+                    if (flags[0] == 0) do {
+                        // ---- A: loads, cumulative log-decay, span, chunk length.
+                        // Warp w owns tokens [8w, 8w+8); lane l owns key channels [4l, 4l+4)
+                        // and, for l < 16, value channels dv0 + [4l, 4l+4).
+                        float *wtot = (float *)(xbuf + L::WT), *probe = (float *)(xbuf + L::PR);
+                        float *spanred = (float *)(xbuf + L::XV), *diagq = spanred + 64, *diagb = spanred + 128;
+                        float *lw = (float *)(xbuf + L::LW), *yb = (float *)(xbuf + L::YB);
+                        const uint32_t s_ti = tc::smem_u32(xbuf + L::TI), s_mm = tc::smem_u32(xbuf + L::MM);
+                        const int tb = 8 * warp, c4 = 4 * lane;
+                        // token u's inputs, loaded one token ahead of their use below so that a
+                        // thread never holds more than two tokens' worth (a register peak here
+                        // would make the whole chain kernel spill)
+                        auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
+                        auto load_la = [&](int u) -> float4 {
+                            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (t0 + tb + u < wend) {
+                                if (p.decay_tok) {
+                                    const float sc = __ldg(p.la + gt_of(u));
+                                    x = make_float4(sc, sc, sc, sc);
+                                } else {
+                                    x = __ldg(reinterpret_cast<const float4 *>(p.la + gt_of(u) * kDK + c4));
+                                }
+                            }
+                            return x;
+                        };
+                        auto load_kq = [&](int u, uint2 (&o)[4]) {        // k, q, z, b: 4 bf16 each
+                            const bool in = t0 + tb + u < wend;
+                            const size_t gt = gt_of(u), gk = gt * kDK + c4;
+                            o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
+                            o[1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
+                            o[2] = in && p.z ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
+                            o[3] = !in ? make_uint2(0, 0)
+                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
+                        };
+                        auto load_vw = [&](int u, uint2 (&o)[2]) {        // v, w of this CTA's value columns
+                            const bool in = t0 + tb + u < wend && c4 < kDVC;
+                            const size_t gt = gt_of(u), gv = gt * kDV + dv0 + c4;
+                            o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
+                            o[1] = !in ? make_uint2(0, 0)
+                                  : p.beta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                        };
+                        // inclusive scan over tokens: this warp's sum (and its prefix at tokens
+                        // 0, 1, 3 and 7 of the warp, the probe tokens it may own), then across warps
+                        float off[4] = {0.f, 0.f, 0.f, 0.f};
+                        {
+                            float run[4] = {0.f, 0.f, 0.f, 0.f}, pre[4][4];
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const float4 x = load_la(u);
+                                run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
+                                const int j = u == 0 ? 0 : u == 1 ? 1 : u == 3 ? 2 : u == 7 ? 3 : -1;
+                                if (j >= 0)
+    #pragma unroll
+                                    for (int c = 0; c < 4; ++c) pre[j][c] = run[c];
+                            }
+                            *reinterpret_cast<float4 *>(wtot + warp * kDK + c4) = make_float4(run[0], run[1], run[2], run[3]);
+                            main_sync();
+                            for (int ww = 0; ww < warp; ++ww) {
+                                const float4 o4 = *reinterpret_cast<const float4 *>(wtot + ww * kDK + c4);
+                                off[0] += o4.x; off[1] += o4.y; off[2] += o4.z; off[3] += o4.w;
+                            }
+                            // Lambda at tokens 0, 1, 3, 7, 15, 31, 63 (the last token of a chunk of 2^j):
+                            // tokens 0-7 are warp 0's, 15 warp 1's, 31 warp 3's, 63 warp 7's last
+                            auto put = [&](int j, int k) {
+                                *reinterpret_cast<float4 *>(probe + j * kDK + c4) =
+                                    make_float4(off[0] + pre[k][0], off[1] + pre[k][1], off[2] + pre[k][2], off[3] + pre[k][3]);
+                            };
+                            if (warp == 0) {
+                                put(0, 0);
+                                put(1, 1);
+                                put(2, 2);
+                                put(3, 3);
+                            } else if (warp == 1) {
+                                put(4, 3);
+                            } else if (warp == 3) {
+                                put(5, 3);
+                            } else if (warp == 7) {
+                                put(6, 3);
+                            }
+                        }
+                        main_sync();
+                        {
+                            // span of a chunk of 2^j tokens: max over this thread's 4 channels, then the CTA
+                            const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
+                            float sp[7];
+    #pragma unroll
+                            for (int j = 0; j < 7; ++j) {
+                                const float4 lj = *reinterpret_cast<const float4 *>(probe + j * kDK + c4);
+                                float m = fmaxf(fmaxf(l0.x - lj.x, l0.y - lj.y), fmaxf(l0.z - lj.z, l0.w - lj.w));
+    #pragma unroll
+                                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                                sp[j] = m;
+                            }
+                            if (lane == 0)
+    #pragma unroll
+                                for (int j = 0; j < 7; ++j) spanred[warp * 8 + j] = sp[j];
+                        }
+                        main_sync();
+                        if (tid == 0) {
+                            int nj = 0;
+                            for (int j = 6; j >= 0; --j) {
+                                float m = 0.f;
+                                for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, spanred[ww * 8 + j]);
+                                if (m <= kSpanMax) { nj = j; break; }
+                            }
+                            flags[1] = min(1 << nj, wend - t0);
+                            flags[2] = nj;
+                        }
+                        const bool vlane = c4 < kDVC;
+                        main_sync();
+                        n = flags[1];
+
+                        // ---- B: operand tiles (fp16, swizzled), pivot vectors, exact diagonals
+                        {
+                            // Lambda_{n-1} is the probe of the chosen power-of-two chunk: past the
+                            // end of the sequence the log-decay is zero-padded, so a shorter tail
+                            // has the same cumulative value there.
+                            const int jn = flags[2];
+                            const float4 l0 = *reinterpret_cast<const float4 *>(probe + c4);
+                            const float4 ln4 = *reinterpret_cast<const float4 *>(probe + jn * kDK + c4);
+                            const float l0v[4] = {l0.x, l0.y, l0.z, l0.w};
+                            const float lnv[4] = {ln4.x, ln4.y, ln4.z, ln4.w};
+                            float cpiv[4], gq[4];
+    #pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                cpiv[c] = 0.5f * (l0v[c] + lnv[c]);
+                                gq[c] = gsv[c4 + c];
+                                if (warp == 0) {
+                                    ecv[c4 + c] = __expf(cpiv[c]);
+                                    fcv[c4 + c] = __expf(lnv[c] - cpiv[c]);
+                                }
+                            }
+                            float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
+                            float4 la_nx = load_la(0);
+                            uint2 kq_nx[4];
+                            load_kq(0, kq_nx);
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int t = tb + u;
+                                const bool live = t < n;
+                                const float4 la_c = la_nx;
+                                const uint2 kq_c[4] = {kq_nx[0], kq_nx[1], kq_nx[2], kq_nx[3]};
+                                if (u + 1 < 8) {
+                                    la_nx = load_la(u + 1);
+                                    load_kq(u + 1, kq_nx);
+                                }
+                                lam_run[0] += la_c.x; lam_run[1] += la_c.y; lam_run[2] += la_c.z; lam_run[3] += la_c.w;
+                                float kk[4], qq[4], zz[4], bv[4];
+                                {
+                                    const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[0]);
+                                    const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[1]);
+                                    const __nv_bfloat162 *hz = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[2]);
+                                    const __nv_bfloat162 *hb = reinterpret_cast<const __nv_bfloat162 *>(&kq_c[3]);
+    #pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        float2 f;
+                                        f = __bfloat1622float2(hk[e]); kk[2 * e] = f.x; kk[2 * e + 1] = f.y;
+                                        f = __bfloat1622float2(hq[e]); qq[2 * e] = f.x; qq[2 * e + 1] = f.y;
+                                        f = __bfloat1622float2(hz[e]); zz[2 * e] = f.x; zz[2 * e + 1] = f.y;
+                                        f = __bfloat1622float2(hb[e]); bv[2 * e] = f.x; bv[2 * e + 1] = f.y;
+                                    }
+                                    if (kRaw) {                 // the q/k preprocessing, one token a call
+                                        silu_l2n_row4(kk);
+                                        silu_l2n_row4(qq);
+                                    }
+                                }
+                                float kp[4], kc[4], khc[4], qp[4];
+                                float dq = 0.f, db = 0.f;
+    #pragma unroll
+                                for (int c = 0; c < 4; ++c) {
+                                    const float lam = live ? lam_run[c] : lnv[c];   // identity padding past n
+                                    const float d = lam - cpiv[c];
+                                    const float ep = __expf(d), em = __expf(-d);
+                                    const float kv = live ? kk[c] : 0.f;
+                                    const float qt = live ? qq[c] * gq[c] * (2.f / (1.f + __expf(-zz[c]))) : 0.f;
+                                    const float kh = bv[c] * kv;
+                                    dq += qt * kv;
+                                    db += qt * kh;
+                                    kp[c] = kv * ep;
+                                    kc[c] = kv * em;
+                                    khc[c] = kh * em;
+                                    qp[c] = qt * ep;
+                                }
+                                range_max = fmaxf(range_max, fmaxf(fmaxf(maxabs(kp, 4), maxabs(kc, 4)),
+                                                                   fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
+                                // the diagonal of Aq / Bq carries no decay: it is summed exactly in
+                                // fp32 (a readout whose q~.k nearly cancels, e.g. the first token of a
+                                // sequence, is then free of fp16 operand rounding)
+    #pragma unroll
+                                for (int o = 16; o > 0; o >>= 1) {
+                                    dq += __shfl_xor_sync(0xffffffffu, dq, o);
+                                    db += __shfl_xor_sync(0xffffffffu, db, o);
+                                }
+                                if (lane == 0) {
+                                    diagq[t] = dq;
+                                    diagb[t] = db;
+                                }
+                                const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
+                                *(uint2 *)(buf + L::AP + off_t) = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
+                                *(uint2 *)(buf + L::AP + off_b) = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
+                                *(uint2 *)(buf + L::BP + off_t) = make_uint2(tc::pack_half2(kc[0], kc[1]), tc::pack_half2(kc[2], kc[3]));
+                                *(uint2 *)(buf + L::BP + off_b) =
+                                    make_uint2(tc::pack_half2(khc[0], khc[1]), tc::pack_half2(khc[2], khc[3]));
+                            }
+                            if (vlane) {
+                                uint2 vw_nx[2];
+                                load_vw(0, vw_nx);
+    #pragma unroll
+                                for (int u = 0; u < 8; ++u) {
+                                    const int t = tb + u;
+                                    const bool live = t < n;
+                                    const uint2 vw_c[2] = {vw_nx[0], vw_nx[1]};
+                                    if (u + 1 < 8) load_vw(u + 1, vw_nx);
+                                    const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
+                                    const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
+                                    float vh[4];
+    #pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        const float2 fv = __bfloat1622float2(hv[e]), fw = __bfloat1622float2(hw[e]);
+                                        vh[2 * e] = live ? fv.x * fw.x : 0.f;
+                                        vh[2 * e + 1] = live ? fv.y * fw.y : 0.f;
+                                    }
+                                    *(uint2 *)(buf + L::VH + tc::tile_off(64, t, c4)) =
+                                        make_uint2(tc::pack_half2(vh[0], vh[1]), tc::pack_half2(vh[2], vh[3]));
+                                }
+                            }
+                        }
+                        tc::fence_proxy_async();
+                        main_sync();
+
+                        // ---- C: decay-relative products P = [Kp; Qp] [Kc; K^c]^T
+                        if (tid == 0) {
+                            tc::fence_after_sync();
+                            const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
+                            for (int ks = 0; ks < kDK / 16; ++ks)
+                                tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id,
+                                            ks > 0);
+                            tc::mma_commit(s_mbar);
+                        }
+                        if (!wait_mma()) break;
+
+                        // ---- D: masks; M -> MM, L -> fp32, Aq/Bq -> ANAB
+                        {
+                            // rows 0-63: warps 0,1 (M, cols 0-63) and warps 4,5 (L, cols 64-127)
+                            // rows 64-127: warps 2,3 (Aq) and warps 6,7 (Bq)
+                            const int t = row & 63;
+                            const bool upper = row < 64;
+                            float v[2][32];
+                            tc::tmem_ld32x2(tmem + lane_base + kTmP + 64 * colhalf, tmem + lane_base + kTmP + 64 * colhalf + 32,
+                                            v[0], v[1]);
+    #pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+    #pragma unroll
+                                for (int i = 0; i < 32; ++i) {
+                                    const int s = 32 * hf + i;
+                                    const bool keep = upper ? (s < t) : (s <= t);
+                                    if (!keep) v[hf][i] = 0.f;
+                                    if (!upper && s == t) v[hf][i] = colhalf == 0 ? diagq[t] : diagb[t];
+                                }
+                                if (upper && colhalf == 1) {
+                                    float4 *dst = reinterpret_cast<float4 *>(lw + t * kLW + 32 * hf);
+    #pragma unroll
+                                    for (int q = 0; q < 8; ++q)
+                                        dst[q] = make_float4(v[hf][4 * q], v[hf][4 * q + 1], v[hf][4 * q + 2], v[hf][4 * q + 3]);
+                                } else {
+                                    uint8_t *tile = upper ? xbuf + L::MM : buf + L::ANAB;
+                                    const int R = upper ? 64 : 192;
+                                    const int r = upper ? t : (colhalf == 0 ? 64 + t : 128 + t);
+                                    store_row32(tile, R, r, 32 * hf, v[hf]);
+                                }
+                            }
+                        }
+                        tc::fence_before_sync();
+                        main_sync();
+
+                        // ---- E: T^-1 = (I + L)^-1 in place, divide and conquer (fp32)
+                        {
+                            // leaves of 8: forward substitution per column, in registers
+                            if (tid < 64) {
+                                const int o = 8 * (tid >> 3), j = tid & 7;
+                                float Lr[8][8];
+    #pragma unroll
+                                for (int i = 1; i < 8; ++i)
+    #pragma unroll
+                                    for (int s = 0; s < i; ++s) Lr[i][s] = lw[(o + i) * kLW + o + s];
+                                float x[8];
+    #pragma unroll
+                                for (int i = 0; i < 8; ++i) x[i] = (i == j) ? 1.f : 0.f;
+    #pragma unroll
+                                for (int i = 1; i < 8; ++i) {
+                                    float acc = 0.f;
+    #pragma unroll
+                                    for (int s = 0; s < i; ++s) acc += Lr[i][s] * x[s];
+                                    if (i > j) x[i] = -acc;
+                                }
+                                __syncwarp();
+                                asm volatile("bar.sync 2, 64;" ::: "memory");     // the 64 leaf threads only
+    #pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    if (i >= j) lw[(o + i) * kLW + o + j] = x[i];
+                            }
+                            main_sync();
+                            // merges: [[A, 0], [C, D]]^-1 = [[A^-1, 0], [-D^-1 C A^-1, D^-1]],
+                            // four output columns per task; the upper triangles are zero, so the
+                            // sums run over whole blocks without masks
+                            merge_level<8>(lw, yb, tid);
+                            merge_level<16>(lw, yb, tid);
+                            merge_level<32>(lw, yb, tid);
+                            // T^-1 -> fp16 tile (row t, column s; the upper part of lw is zero)
+                            for (int u = tid; u < 64 * 8; u += kThreads) {
+                                const int t = u >> 3, g8 = u & 7;
+                                const float4 a = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8);
+                                const float4 b4 = *reinterpret_cast<const float4 *>(lw + t * kLW + 8 * g8 + 4);
+                                const float f[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
+                                *(uint4 *)(xbuf + L::TI + tc::tile_chunk_off(64, t, g8)) = pack8(f);
+                            }
+                        }
+                        tc::fence_proxy_async();
+                        main_sync();
+
+                        // ---- F: W' = T^-1 Kp, N = T^-1 M
+                        if (tid == 0) {
+                            tc::fence_after_sync();
+                            const uint32_t idw = tc::idesc_f16(64, 128, false, true, false);
+                            const uint32_t idn = tc::idesc_f16(64, 64, false, true, false);
+                            for (int ks = 0; ks < kC / 16; ++ks)
+                                tc::mma_f16(tmem + kTmW, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_ap, 128, 0, ks), idw,
+                                            ks > 0);
+                            for (int ks = 0; ks < kC / 16; ++ks)
+                                tc::mma_f16(tmem + kTmN, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_mm, 64, 0, ks), idn,
+                                            ks > 0);
+                            tc::mma_commit(s_mbar);
+                        }
+                        if (!wait_mma()) break;
+
+                        // ---- G: W' -> rows 0-63 of AP (over Kp), N -> rows 0-63 of ANAB.
+                        // M = 64 accumulators sit in lanes 0-15 of each 32-lane group.
+                        {
+                            const int t = 16 * (warp & 3) + lane;
+                            const bool valid = lane < 16;
+                            float v[2][32];
+                            // warps 0-3: W' columns 0-63; warps 4-7: W' columns 64-127
+                            tc::tmem_ld32x2(tmem + lane_base + kTmW + 64 * colhalf, tmem + lane_base + kTmW + 64 * colhalf + 32,
+                                            v[0], v[1]);
+                            if (valid) {
+    #pragma unroll
+                                for (int hf = 0; hf < 2; ++hf) {
+                                    range_max = fmaxf(range_max, maxabs(v[hf], 32));
+                                    store_row32(buf + L::AP, 128, t, 64 * colhalf + 32 * hf, v[hf]);
+                                }
+                            }
+                            // warps 0-3: N columns 0-31; warps 4-7: N columns 32-63
+                            float nv[32];
+                            tc::tmem_ld32(tmem + lane_base + kTmN + 32 * colhalf, nv);
+                            if (valid) {
+                                range_max = fmaxf(range_max, maxabs(nv, 32));
+                                store_row32(buf + L::ANAB, 192, t, 32 * colhalf, nv);
+                            }
+                        }
+                    } while (false);
+                    chunk_products(t0, n);
+                    t0 += n;
+                }
             }
             // after a window processed in shorter chunks: the record of window w + 1
             // (its scratch buffer) is copied again, and this buffer takes window w + 2
