@@ -16,13 +16,16 @@
 // 16-bit operands; one bf16 part alone would round them to 8 bits, which the
 // log-decay's sensitivity to its logit shows (about 4 % of its rms on the
 // workload), while the two parts carry about 16 bits.
-// A CTA runs one SM: warp 0 stages A and B tiles with TMA into a 4-deep ring
-// (128-byte swizzle, the layout the MMA descriptors read), warp 1 issues the
-// MMAs (M = 128 tokens, N = 256 columns, K = 64 per stage) into one of two
-// TMEM accumulators, warps 2-9 drain the other accumulator (bias, activation,
-// stores) meanwhile: two warps per 32-lane TMEM quadrant, one per half of the
-// tile's columns.
+// A CTA runs one SM: warp 0 stages A and B tiles with TMA into a ring of
+// stages (128-byte swizzle, the layout the MMA descriptors read), warp 1 issues
+// the MMAs (M = 128 tokens, N = 256 columns, K = 64 per stage) into one of two
+// TMEM accumulators, warps 2-9 drain the other accumulator meanwhile: two warps
+// per 32-lane TMEM quadrant, one per half of the tile's columns.  The down
+// launch stores the code halves directly; the up launch adds the bias, applies
+// the activation and writes the gates through shared memory with TMA stores
+// (one instruction per 4 KB box instead of 16-byte stores to 32 rows).
 #include <cuda.h>
+#include <cstring>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -35,45 +38,58 @@ namespace {
 constexpr int kPM = 128;                          // tokens per tile
 constexpr int kPN = 256;                          // output columns per tile
 constexpr int kPK = 64;                           // contraction per stage (128 bytes of bf16)
-constexpr int kPStages = 4;
 constexpr int kPATile = kPM * kPK * 2;            // 16 KiB
 constexpr int kPBTile = kPK * kPN * 2;            // 32 KiB: 4 column blocks of 64 x 64
 constexpr int kPStage = kPATile + kPBTile;
 constexpr int kPThreads = 320;                   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int kPEpiWarps = 8;
+constexpr int kPBox = 32 * 128;                   // one staged output box: 32 rows of 128 bytes
 constexpr uint32_t kPDrainPolls = 1u << 22;
 
+// Shared memory.  down: a 4-deep operand ring.  up: a 3-deep ring, two staged
+// output boxes per epilogue warp (1024-byte aligned, as the 128-byte swizzle
+// wants) and each epilogue warp's slice of the bias (128 floats).
+template <bool kUp>
 struct ProjSmem {
+    static constexpr int kStages = kUp ? 3 : 4;
     static constexpr int STAGES = 0;
-    static constexpr int BAR = kPStages * kPStage;             // full[4], empty[4], acc_full[2], acc_empty[2], stall
-    static constexpr int MISC = BAR + 8 * (2 * kPStages + 5);  // TMEM slot, abort flag
+    static constexpr int OUT = kStages * kPStage;
+    static constexpr int BIAS = OUT + (kUp ? kPEpiWarps * 2 * kPBox : 0);
+    static constexpr int BAR = BIAS + (kUp ? kPEpiWarps * 128 * 4 : 0);  // full, empty, acc_full[2], acc_empty[2], stall
+    static constexpr int MISC = BAR + 8 * (2 * kStages + 5);              // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 64;
+    static_assert(OUT % 1024 == 0, "staged boxes start on a 1024-byte boundary");
 };
 
 struct ProjParams {
     int M;                 // tokens
     int d;                 // model width
     int R;                 // total rank
-    int up;                // 0: codes = x w_down; 1: gate logits -> activations
     int jobs;              // output tiles
     int nn;                // column tiles per (token tile, gate)
     int rk[5], roff[5];    // ranks and their offsets in the code
-    __nv_bfloat16 *codes;  // [M, 2R]: hi | lo
-    float *log_alpha;      // [M, d]
-    __nv_bfloat16 *gb, *gg, *gw, *gz;
+    __nv_bfloat16 *codes;  // [M, 2R]: hi | lo (written by the down launch)
     const float *bias;     // [5, d]
     int *status;
     uint32_t spin;
     int stall;             // failure-path test: wait first on a barrier nothing completes
 };
 
+// The up launch's outputs as TMA store maps (128-byte swizzle): log alpha
+// [M, d] fp32 in boxes of 32 columns x 32 rows, b, g, w, z [M, d] bf16 in boxes
+// of 64 columns x 32 rows.
+struct OutMaps {
+    CUtensorMap la, gb, gg, gw, gz;
+};
+
 struct Job {
     int m0, n0, k0, nk, gate;
 };
 
+template <bool kUp>
 __device__ __forceinline__ Job job_of(const ProjParams &p, int j) {
     Job t;
-    if (!p.up) {
+    if (!kUp) {
         t.m0 = kPM * (j / p.nn);
         t.n0 = kPN * (j % p.nn);
         t.k0 = 0;
@@ -121,11 +137,18 @@ __device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 }  // namespace
 
+template <bool kUp>
 __global__ void __launch_bounds__(kPThreads, 1)
-    gate_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, ProjParams p) {
-    using L = ProjSmem;
+    gate_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ OutMaps om, const __grid_constant__ ProjParams p) {
+    using L = ProjSmem<kUp>;
+    constexpr int kPStages = L::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -165,7 +188,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // ---- TMA producer
         uint32_t it = 0;
         for (int j = blockIdx.x; j < p.jobs && !timed_out; j += gridDim.x) {
-            const Job t = job_of(p, j);
+            const Job t = job_of<kUp>(p, j);
             for (int kk = 0; kk < t.nk; ++kk, ++it) {
                 const uint32_t s = it % kPStages, u = it / kPStages;
                 if (*abort_flag || (u > 0 && !tc::mbar_wait(s_empty + 8 * s, (u - 1) & 1u, p.spin))) {
@@ -174,7 +197,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 }
                 // up: the second half of the stages reads the lo part of the codes
                 // against the same rows of w_up
-                const int half = p.up ? t.nk / 2 : t.nk;
+                const int half = kUp ? t.nk / 2 : t.nk;
                 const int kr = kk % half, ka = t.k0 + kPK * kr + (kk >= half ? p.R : 0);
                 const uint32_t a = tc::smem_u32(sm + L::STAGES + s * kPStage), b = a + kPATile;
                 tc::mbar_arrive_expect_tx(s_full + 8 * s, kPStage);
@@ -197,7 +220,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         uint32_t it = 0, t = 0;
         bool issued = false;
         for (int j = blockIdx.x; j < p.jobs && !timed_out; j += gridDim.x, ++t) {
-            const Job jb = job_of(p, j);
+            const Job jb = job_of<kUp>(p, j);
             const uint32_t b = t & 1u, v = t >> 1;
             if (*abort_flag || (v > 0 && !tc::mbar_wait(s_acce + 8 * b, (v - 1) & 1u, p.spin))) {
                 timed_out = true;
@@ -231,13 +254,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 tc::mbar_wait(s_empty + 8 * (last % kPStages), (last / kPStages) & 1u, kPDrainPolls);
             }
         }
-    } else if (warp >= 2) {
-        // ---- epilogue: TMEM lanes 32 (warp % 4) .. +31 are the tile's rows; warps
-        // 2-5 take columns 0-127 of the tile, warps 6-9 columns 128-255
+    } else if (warp >= 2 && !kUp) {
+        // ---- down epilogue: TMEM lanes 32 (warp % 4) .. +31 are the tile's rows;
+        // warps 2-5 take columns 0-127 of the tile, warps 6-9 columns 128-255
         const int qd = warp & 3, row = 32 * qd + lane, cbase = warp < 6 ? 0 : kPN / 2;
         uint32_t t = 0;
         for (int j = blockIdx.x; j < p.jobs; j += gridDim.x, ++t) {
-            const Job jb = job_of(p, j);
+            const Job jb = job_of<kUp>(p, j);
             const uint32_t b = t & 1u, v = t >> 1;
             bool ok = true;
             if (lane == 0) ok = !*abort_flag && tc::mbar_wait(s_accf + 8 * b, v & 1u, p.spin);
@@ -249,59 +272,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
             tc::fence_after_sync();
             const uint32_t acc = tmem + ((uint32_t)(32 * qd) << 16) + b * kPN;
             const int m = jb.m0 + row;
-            const bool live = m < p.M;
             for (int c = 0; c < kPN / 64; ++c) {
                 float x[32];
                 tc::tmem_ld32(acc + cbase + 32 * c, x);
                 const int n = jb.n0 + cbase + 32 * c;
-                if (!p.up) {
-                    if (live) {
-                        // c = hi + lo: hi its bf16 rounding, lo the bf16 rounding of the rest
-                        float lo[32];
+                if (m < p.M) {
+                    // c = hi + lo: hi its bf16 rounding, lo the bf16 rounding of the rest
+                    float lo[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) lo[i] = x[i] - __bfloat162float(__float2bfloat16_rn(x[i]));
-                        uint4 *dh = reinterpret_cast<uint4 *>(p.codes + (size_t)m * 2 * p.R + n);
-                        uint4 *dl = reinterpret_cast<uint4 *>(p.codes + (size_t)m * 2 * p.R + p.R + n);
+                    for (int i = 0; i < 32; ++i) lo[i] = x[i] - __bfloat162float(__float2bfloat16_rn(x[i]));
+                    uint4 *dh = reinterpret_cast<uint4 *>(p.codes + (size_t)m * 2 * p.R + n);
+                    uint4 *dl = reinterpret_cast<uint4 *>(p.codes + (size_t)m * 2 * p.R + p.R + n);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            dh[q] = make_uint4(pack_bf2(x[8 * q], x[8 * q + 1]), pack_bf2(x[8 * q + 2], x[8 * q + 3]),
-                                               pack_bf2(x[8 * q + 4], x[8 * q + 5]), pack_bf2(x[8 * q + 6], x[8 * q + 7]));
-                            dl[q] = make_uint4(pack_bf2(lo[8 * q], lo[8 * q + 1]), pack_bf2(lo[8 * q + 2], lo[8 * q + 3]),
-                                               pack_bf2(lo[8 * q + 4], lo[8 * q + 5]), pack_bf2(lo[8 * q + 6], lo[8 * q + 7]));
-                        }
+                    for (int q = 0; q < 4; ++q) {
+                        dh[q] = make_uint4(pack_bf2(x[8 * q], x[8 * q + 1]), pack_bf2(x[8 * q + 2], x[8 * q + 3]),
+                                           pack_bf2(x[8 * q + 4], x[8 * q + 5]), pack_bf2(x[8 * q + 6], x[8 * q + 7]));
+                        dl[q] = make_uint4(pack_bf2(lo[8 * q], lo[8 * q + 1]), pack_bf2(lo[8 * q + 2], lo[8 * q + 3]),
+                                           pack_bf2(lo[8 * q + 4], lo[8 * q + 5]), pack_bf2(lo[8 * q + 6], lo[8 * q + 7]));
                     }
-                    continue;
-                }
-                const float *bias = p.bias + (size_t)jb.gate * p.d + n;
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 bv = __ldg(reinterpret_cast<const float4 *>(bias + i));
-                    x[i] += bv.x;
-                    x[i + 1] += bv.y;
-                    x[i + 2] += bv.z;
-                    x[i + 3] += bv.w;
-                }
-                if (!live) continue;
-                if (jb.gate == 0) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.log_alpha + (size_t)m * p.d + n);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(plogsigmoid(x[4 * q]), plogsigmoid(x[4 * q + 1]), plogsigmoid(x[4 * q + 2]),
-                                             plogsigmoid(x[4 * q + 3]));
-                } else {
-                    __nv_bfloat16 *out = jb.gate == 1 ? p.gb : jb.gate == 2 ? p.gg : jb.gate == 3 ? p.gw : p.gz;
-                    if (jb.gate == 1) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] = 2.f * psigmoid(x[i]);
-                    } else if (jb.gate != 4) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] = psigmoid(x[i]);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)m * p.d + n);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pack_bf2(x[8 * q], x[8 * q + 1]), pack_bf2(x[8 * q + 2], x[8 * q + 3]),
-                                            pack_bf2(x[8 * q + 4], x[8 * q + 5]), pack_bf2(x[8 * q + 6], x[8 * q + 7]));
                 }
             }
             // this warp's reads of the accumulator are complete: hand it back
@@ -309,6 +297,107 @@ __global__ void __launch_bounds__(kPThreads, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive_local(s_acce + 8 * b);
         }
+        if (timed_out && lane == 0) *abort_flag = 1;
+    } else if (warp >= 2) {
+        // ---- up epilogue.  The warp owns TMEM lanes 32 (warp % 4) .. +31 (the
+        // tile's rows) and 128 of its columns (warps 2-5 the first half, 6-9 the
+        // second).  Activated values are staged in shared memory as boxes of 32
+        // rows x 128 bytes (32 fp32 or 64 bf16 columns), each row's 16-byte chunks
+        // in the 128-byte-swizzled order (chunk q at q ^ (row % 8): the eight rows
+        // a store phase covers hit eight different bank groups), and lane 0 writes
+        // each box with one TMA store; two boxes per warp alternate.
+        const int ew = warp - 2, qd = warp & 3, cbase = warp < 6 ? 0 : kPN / 2;
+        const uint32_t obuf = tc::smem_u32(sm + L::OUT + ew * 2 * kPBox);
+        float *sbias = reinterpret_cast<float *>(sm + L::BIAS + ew * 128 * 4);
+        const uint32_t rowoff = (uint32_t)lane * 128u, sw = (uint32_t)(lane & 7);
+        uint32_t t = 0, nbox = 0;
+        for (int j = blockIdx.x; j < p.jobs; j += gridDim.x, ++t) {
+            const Job jb = job_of<kUp>(p, j);
+            const uint32_t b = t & 1u, v = t >> 1;
+            // this warp's 128 bias values, fetched before the accumulator wait
+            const float4 bv =
+                __ldg(reinterpret_cast<const float4 *>(p.bias + (size_t)jb.gate * p.d + jb.n0 + cbase) + lane);
+            bool ok = true;
+            if (lane == 0) ok = !*abort_flag && tc::mbar_wait(s_accf + 8 * b, v & 1u, p.spin);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                timed_out = true;
+                break;
+            }
+            tc::fence_after_sync();
+            const uint32_t acc = tmem + ((uint32_t)(32 * qd) << 16) + b * kPN + cbase;
+            const int y = jb.m0 + 32 * qd;                 // the boxes' first row
+            auto release = [&]() {
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive_local(s_acce + 8 * b);
+            };
+            if (y >= p.M) {                                // rows past the last token: nothing to store
+                release();
+                continue;
+            }
+            reinterpret_cast<float4 *>(sbias)[lane] = bv;
+            __syncwarp();
+            const CUtensorMap *map = jb.gate == 0 ? &om.la : jb.gate == 1 ? &om.gb : jb.gate == 2 ? &om.gg
+                                     : jb.gate == 3 ? &om.gw : &om.gz;
+            const int cols = jb.gate == 0 ? 32 : 64;       // columns per box
+            for (int bx = 0; bx < 128 / cols; ++bx, ++nbox) {
+                // the buffer was last read by the store two boxes back
+                if (lane == 0) tc::bulk_wait_read_n<1>();
+                __syncwarp();
+                const uint32_t buf = obuf + (nbox & 1u) * kPBox + rowoff;
+                if (jb.gate == 0) {
+                    float x[32];
+                    tc::tmem_ld32(acc + 32 * bx, x);
+                    if (bx == 3) release();
+                    const float4 *bb = reinterpret_cast<const float4 *>(sbias + 32 * bx);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 c4 = bb[q];
+                        st_shared_v4(buf + ((q ^ sw) << 4), __float_as_uint(plogsigmoid(x[4 * q] + c4.x)),
+                                     __float_as_uint(plogsigmoid(x[4 * q + 1] + c4.y)),
+                                     __float_as_uint(plogsigmoid(x[4 * q + 2] + c4.z)),
+                                     __float_as_uint(plogsigmoid(x[4 * q + 3] + c4.w)));
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float x[32];
+                        tc::tmem_ld32(acc + 64 * bx + 32 * h, x);
+                        if (bx == 1 && h == 1) release();
+                        const float4 *bb = reinterpret_cast<const float4 *>(sbias + 64 * bx + 32 * h);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 c4 = bb[q];
+                            x[4 * q] += c4.x;
+                            x[4 * q + 1] += c4.y;
+                            x[4 * q + 2] += c4.z;
+                            x[4 * q + 3] += c4.w;
+                        }
+                        if (jb.gate == 1) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) x[i] = 2.f * psigmoid(x[i]);
+                        } else if (jb.gate != 4) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) x[i] = psigmoid(x[i]);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            st_shared_v4(buf + (((uint32_t)(4 * h + q) ^ sw) << 4), pack_bf2(x[8 * q], x[8 * q + 1]),
+                                         pack_bf2(x[8 * q + 2], x[8 * q + 3]), pack_bf2(x[8 * q + 4], x[8 * q + 5]),
+                                         pack_bf2(x[8 * q + 6], x[8 * q + 7]));
+                    }
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::tma_store_2d(map, obuf + (nbox & 1u) * kPBox, jb.n0 + cbase + cols * bx, y);
+                    tc::bulk_commit();
+                }
+            }
+        }
+        // the boxes' stores are complete before the CTA's shared memory goes away
+        if (lane == 0) tc::bulk_wait_all();
         if (timed_out && lane == 0) *abort_flag = 1;
     }
     tc::fence_before_sync();
@@ -340,17 +429,32 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A row-major [rows, cols] bf16 matrix, boxes of 64 columns x box_rows rows.
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// A row-major [rows, cols] matrix of `esize`-byte elements, boxes of box_cols x
+// box_rows with the 128-byte swizzle (box_cols * esize = 128).
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize, uint64_t rows, uint64_t cols,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapL2promotion l2) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint64_t strides[1] = {cols * esize};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An operand: bf16, boxes of 64 columns x box_rows rows.
+bool operand_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 64, box_rows,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
+// An output of the up launch: 32 rows of 128 bytes per box.
+bool output_map(CUtensorMap *m, void *base, bool fp32, uint64_t rows, uint64_t cols) {
+    return fp32 ? make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols, 32, 32,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE)
+                : make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 64, 32,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 }  // namespace
@@ -367,8 +471,10 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
         e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
-    const int smem = ProjSmem::TOTAL + 1024;
-    e = cudaFuncSetAttribute(gate_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem_down = ProjSmem<false>::TOTAL + 1024, smem_up = ProjSmem<true>::TOTAL + 1024;
+    e = cudaFuncSetAttribute(gate_proj_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_down);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gate_proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_up);
     if (e != cudaSuccess) return e;
 
     ProjParams p{};
@@ -381,11 +487,6 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
         p.R += gp.ranks[i];
     }
     p.codes = (__nv_bfloat16 *)gp.codes;
-    p.log_alpha = gp.log_alpha;
-    p.gb = (__nv_bfloat16 *)gp.b;
-    p.gg = (__nv_bfloat16 *)gp.g;
-    p.gw = (__nv_bfloat16 *)gp.w;
-    p.gz = (__nv_bfloat16 *)gp.z;
     p.bias = gp.bias;
     p.status = gp.status;
     p.spin = gp.wait_limit;
@@ -393,24 +494,27 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
     const int mt = (gp.N + kPM - 1) / kPM;
 
     CUtensorMap ta, tb;
+    OutMaps om;
+    memset(&om, 0, sizeof(om));                      // the down launch stores directly
     // down: A = x [N, d], B = w_down [d, R]
-    if (!make_map(&ta, gp.x, (uint64_t)gp.N, (uint64_t)gp.d, kPM) ||
-        !make_map(&tb, gp.w_down, (uint64_t)gp.d, (uint64_t)p.R, kPK))
+    if (!operand_map(&ta, gp.x, (uint64_t)gp.N, (uint64_t)gp.d, kPM) ||
+        !operand_map(&tb, gp.w_down, (uint64_t)gp.d, (uint64_t)p.R, kPK))
         return cudaErrorInvalidValue;
-    p.up = 0;
     p.nn = p.R / kPN;
     p.jobs = mt * p.nn;
-    gate_proj_kernel<<<min(sms[dev], p.jobs), kPThreads, smem, stream>>>(ta, tb, p);
+    gate_proj_kernel<false><<<min(sms[dev], p.jobs), kPThreads, smem_down, stream>>>(ta, tb, om, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // up: A = codes [N, 2R] (hi | lo), B = w_up [R, d]
-    if (!make_map(&ta, gp.codes, (uint64_t)gp.N, (uint64_t)(2 * p.R), kPM) ||
-        !make_map(&tb, gp.w_up, (uint64_t)p.R, (uint64_t)gp.d, kPK))
+    // up: A = codes [N, 2R] (hi | lo), B = w_up [R, d]; the five outputs
+    const uint64_t N = (uint64_t)gp.N, d = (uint64_t)gp.d;
+    if (!operand_map(&ta, gp.codes, N, (uint64_t)(2 * p.R), kPM) ||
+        !operand_map(&tb, gp.w_up, (uint64_t)p.R, d, kPK) || !output_map(&om.la, gp.log_alpha, true, N, d) ||
+        !output_map(&om.gb, gp.b, false, N, d) || !output_map(&om.gg, gp.g, false, N, d) ||
+        !output_map(&om.gw, gp.w, false, N, d) || !output_map(&om.gz, gp.z, false, N, d))
         return cudaErrorInvalidValue;
-    p.up = 1;
     p.nn = gp.d / kPN;
     p.jobs = mt * 5 * p.nn;
-    gate_proj_kernel<<<min(sms[dev], p.jobs), kPThreads, smem, stream>>>(ta, tb, p);
+    gate_proj_kernel<true><<<min(sms[dev], p.jobs), kPThreads, smem_up, stream>>>(ta, tb, om, p);
     return cudaGetLastError();
 }
 

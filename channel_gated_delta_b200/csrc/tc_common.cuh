@@ -267,6 +267,24 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap,
         : "memory");
 }
 
+// 2-D tiled TMA store of one box from this CTA's shared memory to the tensor
+// map's global memory (bulk-group completion: bulk_commit, then
+// bulk_wait_read_n / bulk_wait_all).  x, y are the box's first column and row,
+// both non-negative, x a multiple of 16 bytes' worth of elements; rows and
+// columns beyond the tensor's extent are not written.  The sources must be made
+// visible to the async proxy first (fence_proxy_async by the writing threads).
+__device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src_smem, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src_smem), "r"(x), "r"(y)
+                 : "memory");
+}
+// Wait until at most N committed bulk-store groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_n() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Hint: bring `bytes` (a multiple of 16) of global memory into L2.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
