@@ -305,7 +305,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // rows x 128 bytes (32 fp32 or 64 bf16 columns), each row's 16-byte chunks
         // in the 128-byte-swizzled order (chunk q at q ^ (row % 8): the eight rows
         // a store phase covers hit eight different bank groups), and lane 0 writes
-        // each box with one TMA store; two boxes per warp alternate.
+        // each box with one TMA store (one bulk group per box); the warp's two
+        // box buffers alternate.
         const int ew = warp - 2, qd = warp & 3, cbase = warp < 6 ? 0 : kPN / 2;
         const uint32_t obuf = tc::smem_u32(sm + L::OUT + ew * 2 * kPBox);
         float *sbias = reinterpret_cast<float *>(sm + L::BIAS + ew * 128 * 4);
@@ -340,59 +341,84 @@ __global__ void __launch_bounds__(kPThreads, 1)
             __syncwarp();
             const CUtensorMap *map = jb.gate == 0 ? &om.la : jb.gate == 1 ? &om.gb : jb.gate == 2 ? &om.gg
                                      : jb.gate == 3 ? &om.gw : &om.gz;
-            const int cols = jb.gate == 0 ? 32 : 64;       // columns per box
-            for (int bx = 0; bx < 128 / cols; ++bx, ++nbox) {
-                // the buffer was last read by the store two boxes back
-                if (lane == 0) tc::bulk_wait_read_n<1>();
-                __syncwarp();
-                const uint32_t buf = obuf + (nbox & 1u) * kPBox + rowoff;
+            // two rounds of 64 columns: both TMEM loads of a round, then one wait;
+            // the log-decay (fp32) fills two boxes of 32 columns per round, the
+            // bf16 gates one box of 64
+            const int x0 = jb.n0 + cbase;
+#pragma unroll 1
+            for (int r = 0; r < 2; ++r) {
+                float va[32], vb[32];
+                tc::tmem_ld32x2(acc + 64 * r, acc + 64 * r + 32, va, vb);
+                if (r == 1) release();
+                const float4 *bb = reinterpret_cast<const float4 *>(sbias + 64 * r);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 c4 = bb[q], d4 = bb[8 + q];
+                    va[4 * q] += c4.x; va[4 * q + 1] += c4.y; va[4 * q + 2] += c4.z; va[4 * q + 3] += c4.w;
+                    vb[4 * q] += d4.x; vb[4 * q + 1] += d4.y; vb[4 * q + 2] += d4.z; vb[4 * q + 3] += d4.w;
+                }
                 if (jb.gate == 0) {
-                    float x[32];
-                    tc::tmem_ld32(acc + 32 * bx, x);
-                    if (bx == 3) release();
-                    const float4 *bb = reinterpret_cast<const float4 *>(sbias + 32 * bx);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        va[i] = plogsigmoid(va[i]);
+                        vb[i] = plogsigmoid(vb[i]);
+                    }
+                    // both buffers: the stores issued before have finished reading them
+                    if (lane == 0) tc::bulk_wait_read_n<0>();
+                    __syncwarp();
+                    const uint32_t ba = obuf + (nbox & 1u) * kPBox, bq = obuf + ((nbox + 1) & 1u) * kPBox;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 c4 = bb[q];
-                        st_shared_v4(buf + ((q ^ sw) << 4), __float_as_uint(plogsigmoid(x[4 * q] + c4.x)),
-                                     __float_as_uint(plogsigmoid(x[4 * q + 1] + c4.y)),
-                                     __float_as_uint(plogsigmoid(x[4 * q + 2] + c4.z)),
-                                     __float_as_uint(plogsigmoid(x[4 * q + 3] + c4.w)));
+                        st_shared_v4(ba + rowoff + ((q ^ sw) << 4), __float_as_uint(va[4 * q]),
+                                     __float_as_uint(va[4 * q + 1]), __float_as_uint(va[4 * q + 2]),
+                                     __float_as_uint(va[4 * q + 3]));
+                        st_shared_v4(bq + rowoff + ((q ^ sw) << 4), __float_as_uint(vb[4 * q]),
+                                     __float_as_uint(vb[4 * q + 1]), __float_as_uint(vb[4 * q + 2]),
+                                     __float_as_uint(vb[4 * q + 3]));
                     }
+                    tc::fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_store_2d(map, ba, x0 + 64 * r, y);
+                        tc::bulk_commit();
+                        tc::tma_store_2d(map, bq, x0 + 64 * r + 32, y);
+                        tc::bulk_commit();
+                    }
+                    nbox += 2;
                 } else {
+                    if (jb.gate == 1) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float x[32];
-                        tc::tmem_ld32(acc + 64 * bx + 32 * h, x);
-                        if (bx == 1 && h == 1) release();
-                        const float4 *bb = reinterpret_cast<const float4 *>(sbias + 64 * bx + 32 * h);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 c4 = bb[q];
-                            x[4 * q] += c4.x;
-                            x[4 * q + 1] += c4.y;
-                            x[4 * q + 2] += c4.z;
-                            x[4 * q + 3] += c4.w;
+                        for (int i = 0; i < 32; ++i) {
+                            va[i] = 2.f * psigmoid(va[i]);
+                            vb[i] = 2.f * psigmoid(vb[i]);
                         }
-                        if (jb.gate == 1) {
+                    } else if (jb.gate != 4) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) x[i] = 2.f * psigmoid(x[i]);
-                        } else if (jb.gate != 4) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) x[i] = psigmoid(x[i]);
+                        for (int i = 0; i < 32; ++i) {
+                            va[i] = psigmoid(va[i]);
+                            vb[i] = psigmoid(vb[i]);
                         }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            st_shared_v4(buf + (((uint32_t)(4 * h + q) ^ sw) << 4), pack_bf2(x[8 * q], x[8 * q + 1]),
-                                         pack_bf2(x[8 * q + 2], x[8 * q + 3]), pack_bf2(x[8 * q + 4], x[8 * q + 5]),
-                                         pack_bf2(x[8 * q + 6], x[8 * q + 7]));
                     }
-                }
-                tc::fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) {
-                    tc::tma_store_2d(map, obuf + (nbox & 1u) * kPBox, jb.n0 + cbase + cols * bx, y);
-                    tc::bulk_commit();
+                    // this buffer was last read by the store two boxes back
+                    if (lane == 0) tc::bulk_wait_read_n<1>();
+                    __syncwarp();
+                    const uint32_t ba = obuf + (nbox & 1u) * kPBox;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        st_shared_v4(ba + rowoff + (((uint32_t)q ^ sw) << 4), pack_bf2(va[8 * q], va[8 * q + 1]),
+                                     pack_bf2(va[8 * q + 2], va[8 * q + 3]), pack_bf2(va[8 * q + 4], va[8 * q + 5]),
+                                     pack_bf2(va[8 * q + 6], va[8 * q + 7]));
+                        st_shared_v4(ba + rowoff + (((uint32_t)(4 + q) ^ sw) << 4), pack_bf2(vb[8 * q], vb[8 * q + 1]),
+                                     pack_bf2(vb[8 * q + 2], vb[8 * q + 3]), pack_bf2(vb[8 * q + 4], vb[8 * q + 5]),
+                                     pack_bf2(vb[8 * q + 6], vb[8 * q + 7]));
+                    }
+                    tc::fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_store_2d(map, ba, x0 + 64 * r, y);
+                        tc::bulk_commit();
+                    }
+                    nbox += 1;
                 }
             }
         }
