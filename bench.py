@@ -602,6 +602,7 @@ def run_gate_proj(args, gd, shape, dev, stream, rank, world):
         "algorithmic_bytes": nbytes, "flops": flops, "tflops": flops / (ms * 1e-3) / 1e12,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "peak_source": kind,
+                     "traffic": recorded_traffic("channel_gated_delta_b200/csrc/gate_proj.cu"),
                      "note": "4 N d R flops at the measured bf16 peak would take less time than the bytes"},
     }
 
