@@ -336,7 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     tc::cluster_sync();
     tc::fence_after_sync();
     const uint32_t tmem = *tslot;
-    uint32_t phase = 0, rphase[2] = {0u, 0u};
+    uint32_t phase = 0;
+    uint32_t rph = 0u;                           // bit b: parity of record buffer b's next copy
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lanes
     const int row = 32 * (warp & 3) + lane;                         // accumulator row (M = 128)
     const int colhalf = warp >> 2;                                  // 32-column half of this CTA's 64
@@ -408,19 +409,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             if (tid == 0 && !tc::mbar_wait(s_stall, 0, p.spin)) flags[0] = 1;
             main_sync();
         }
-        int loaded[2] = {-1, -1};                     // window whose record buffer b holds or receives
-        bool inflight[2] = {false, false};            // a copy into buffer b not yet waited for
+        // Per record buffer b (0 or 1; selected by value, not by index, so that
+        // nothing lives in local memory): the window it holds or receives, and
+        // whether a copy into it has not been waited for (bit b of infl).
+        int loaded0 = -1, loaded1 = -1;
+        uint32_t infl = 0u;
+        auto loaded_of = [&](int b) -> int { return b ? loaded1 : loaded0; };
+        auto set_loaded = [&](int b, int v) {
+            if (b) loaded1 = v;
+            else loaded0 = v;
+        };
         for (int b = 0; b < 2 && flags[0] == 0; ++b)
             if (win_fast(b)) {
                 if (tid == 0) enqueue(b, b);
-                loaded[b] = b;
-                inflight[b] = true;
+                set_loaded(b, b);
+                infl |= 1u << b;
             }
 
         const size_t sbase = (size_t)head * kDK * kDV;
         bool first = true;
         int chunk = 0;
-        uint32_t uses[2] = {0u, 0u};
+        uint32_t uses0 = 0u, uses1 = 0u;                // chunks that used [R; O] slot 0 / 1
         for (int w = 0; w < NW && flags[0] == 0; ++w) {
             const int B = w & 1;
             uint8_t *buf = sm + B * L::BUF, *xbuf = sm + (B ^ 1) * L::BUF;
@@ -428,22 +437,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             const uint32_t s_anab = tc::smem_u32(buf + L::ANAB), s_vh = tc::smem_u32(buf + L::VH);
             float *ecv = (float *)(buf + L::EV), *fcv = ecv + 128;
             const int wend = min(T, kC * (w + 1));
-            const bool fast = loaded[B] == w;
+            const bool fast = loaded_of(B) == w;
             // tile flag of window w + 2, loaded now and first compared once the window's
             // products are done, so that its latency is hidden
             const int wflag2 = (p.ws != nullptr && w + 2 < NW) ? __ldg(p.wflags + wbase + w + 2) : 1;
             // an abort agreed by the readout warps becomes this group's abort at the barrier below
             if (tid == 0 && flags[3] != 0) flags[0] = 1;
             if (fast) {
-                if (!tc::mbar_wait(s_rbar + 8u * B, rphase[B], p.spin)) flags[0] = 1;
-                rphase[B] ^= 1u;
-                inflight[B] = false;
-            } else if (inflight[B ^ 1]) {
+                if (!tc::mbar_wait(s_rbar + 8u * B, (rph >> B) & 1u, p.spin)) flags[0] = 1;
+                rph ^= 1u << B;
+                infl &= ~(1u << B);
+            } else if ((infl >> (B ^ 1)) & 1u) {
                 // the other buffer is this window's scratch: a record arriving there
                 // lands first, and is copied again after the window
-                if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), rphase[B ^ 1], p.spin)) flags[0] = 1;
-                rphase[B ^ 1] ^= 1u;
-                inflight[B ^ 1] = false;
+                if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), (rph >> (B ^ 1)) & 1u, p.spin)) flags[0] = 1;
+                rph ^= 1u << (B ^ 1);
+                infl &= ~(1u << (B ^ 1));
             }
             main_sync();
             // The products of one chunk (H to K) on the tiles in `buf`.  Called from two
@@ -492,7 +501,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     // ---- I: [R; O] = [W'; Qp] S_c + [N; Aq] V^ ;  X += Kc^T V^
                     if (tid == 0) {
                         // the slot's previous O has been read out of TMEM (and its chunk info)
-                        if (uses[slot] > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u, p.spin))
+                        const uint32_t us = slot ? uses1 : uses0;
+                        if (us > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (us - 1) & 1u, p.spin))
                             flags[0] = 1;
                         // the readout warps learn the chunk's tokens now (to fetch the gate early)
                         info[4 * slot] = t0;
@@ -553,10 +563,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         if (t0 + n == wend) {
                             if (wflag2 == 0) {
                                 if (tid == 0) enqueue(w + 2, B);
-                                loaded[B] = w + 2;
-                                inflight[B] = true;
+                                set_loaded(B, w + 2);
+                                infl |= 1u << B;
                             } else {
-                                loaded[B] = -1;
+                                set_loaded(B, -1);
                             }
                         }
                     }
@@ -565,7 +575,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 tc::fence_before_sync();
                 main_sync();
                 tc::fence_after_sync();
-                ++uses[slot];
+                if (slot) ++uses1;
+                else ++uses0;
             };
             if (fast) {
                 if (flags[0] == 0) chunk_products(kC * w, wend - kC * w);
@@ -939,9 +950,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             // after a window processed in shorter chunks: the record of window w + 1
             // (its scratch buffer) is copied again, and this buffer takes window w + 2
             if (!fast && flags[0] == 0) {
-                if (loaded[B ^ 1] == w + 1) {
+                if (loaded_of(B ^ 1) == w + 1) {
                     if (tid == 0) enqueue(w + 1, B ^ 1);
-                    inflight[B ^ 1] = true;
+                    infl |= 1u << (B ^ 1);
                 }
             }
         }
@@ -949,14 +960,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         // no more chunks: tell the readout warps
         if (tid == 0) {
             const uint32_t slot = (uint32_t)(chunk & 1);
-            if (uses[slot] > 0) tc::mbar_wait(s_fbar + 8u * slot, (uses[slot] - 1) & 1u, p.spin);
+            const uint32_t us = slot ? uses1 : uses0;
+            if (us > 0) tc::mbar_wait(s_fbar + 8u * slot, (us - 1) & 1u, p.spin);
             info[4 * slot + 2] = 1;
             tc::mbar_arrive_local(s_ibar + 8u * slot);
         }
         if (tid == 0) enqueue(-1, 0);
         // copies still in flight (the loop ended early) complete before exit
         for (int b = 0; b < 2; ++b)
-            if (inflight[b]) tc::mbar_wait(s_rbar + 8u * b, rphase[b], kDrainPolls);
+            if ((infl >> b) & 1u) tc::mbar_wait(s_rbar + 8u * b, (rph >> b) & 1u, kDrainPolls);
 
         // ---- S_out = Diag(fprev) X
         if (flags[0] == 0 && p.S_out && T > 0) {
