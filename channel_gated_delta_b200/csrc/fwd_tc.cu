@@ -512,11 +512,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         tc::fence_after_sync();
                         const uint32_t id1 = tc::idesc_f16(128, kDVC, false, true, false);
                         if (flags[0] == 0) {
+#pragma unroll
                             for (int ks = 0; ks < kDK / 16; ++ks)
-                                tc::mma_f16(tmem + ro, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_mnmajor(s_sc, 128, 0, ks),
+                                tc::mma_f16(tmem + ro, tc::desc_kmajor_step(tc::desc_kmajor(s_ap, 128, 0, 0), 128, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_sc, 128, 0, 0), ks),
                                             id1, ks > 0);
+#pragma unroll
                             for (int ks = 0; ks < kC / 16; ++ks)
-                                tc::mma_f16(tmem + ro, tc::desc_kmajor(s_anab, 192, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks),
+                                tc::mma_f16(tmem + ro, tc::desc_kmajor_step(tc::desc_kmajor(s_anab, 192, 0, 0), 192, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_vh, 64, 0, 0), ks),
                                             id1, true);
                         }
                         tc::mma_commit(s_mbar);                   // [R; O]: R is read out next
@@ -524,8 +526,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         // (the next commit covers it)
                         const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, false);
                         if (flags[0] == 0)
+#pragma unroll
                             for (int ks = 0; ks < kC / 16; ++ks)
-                                tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 0, ks), tc::desc_mnmajor(s_vh, 64, 0, ks),
+                                tc::mma_f16(tmem + kTmX, tc::desc_mnmajor_step(tc::desc_mnmajor(s_bp, 128, 0, 0), ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_vh, 64, 0, 0), ks),
                                             id2, true);
                     }
                 }
@@ -545,12 +548,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                     if (tid == 0) {
                         tc::fence_after_sync();
                         const uint32_t id1 = tc::idesc_f16(128, kDVC, false, true, true);
+#pragma unroll
                         for (int ks = 0; ks < kC / 16; ++ks)
-                            tc::mma_f16(tmem + ro, tc::desc_kmajor(s_anab, 192, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks),
+                            tc::mma_f16(tmem + ro, tc::desc_kmajor_step(tc::desc_kmajor(s_anab, 192, 64, 0), 192, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_rr, 64, 0, 0), ks),
                                         id1, true);
                         const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, true);
+#pragma unroll
                         for (int ks = 0; ks < kC / 16; ++ks)
-                            tc::mma_f16(tmem + kTmX, tc::desc_mnmajor(s_bp, 128, 64, ks), tc::desc_mnmajor(s_rr, 64, 0, ks),
+                            tc::mma_f16(tmem + kTmX, tc::desc_mnmajor_step(tc::desc_mnmajor(s_bp, 128, 64, 0), ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_rr, 64, 0, 0), ks),
                                         id2, true);
                         tc::mma_commit(s_mbar);
                         tc::mma_commit(s_obar + 8u * slot);      // O of this chunk is final
@@ -817,8 +822,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         if (tid == 0) {
                             tc::fence_after_sync();
                             const uint32_t id = tc::idesc_f16(128, 128, false, false, false);
+#pragma unroll
                             for (int ks = 0; ks < kDK / 16; ++ks)
-                                tc::mma_f16(tmem + kTmP, tc::desc_kmajor(s_ap, 128, 0, ks), tc::desc_kmajor(s_bp, 128, 0, ks), id,
+                                tc::mma_f16(tmem + kTmP, tc::desc_kmajor_step(tc::desc_kmajor(s_ap, 128, 0, 0), 128, ks), tc::desc_kmajor_step(tc::desc_kmajor(s_bp, 128, 0, 0), 128, ks), id,
                                             ks > 0);
                             tc::mma_commit(s_mbar);
                         }
@@ -908,11 +914,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                             tc::fence_after_sync();
                             const uint32_t idw = tc::idesc_f16(64, 128, false, true, false);
                             const uint32_t idn = tc::idesc_f16(64, 64, false, true, false);
+#pragma unroll
                             for (int ks = 0; ks < kC / 16; ++ks)
-                                tc::mma_f16(tmem + kTmW, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_ap, 128, 0, ks), idw,
+                                tc::mma_f16(tmem + kTmW, tc::desc_kmajor_step(tc::desc_kmajor(s_ti, 64, 0, 0), 64, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_ap, 128, 0, 0), ks), idw,
                                             ks > 0);
+#pragma unroll
                             for (int ks = 0; ks < kC / 16; ++ks)
-                                tc::mma_f16(tmem + kTmN, tc::desc_kmajor(s_ti, 64, 0, ks), tc::desc_mnmajor(s_mm, 64, 0, ks), idn,
+                                tc::mma_f16(tmem + kTmN, tc::desc_kmajor_step(tc::desc_kmajor(s_ti, 64, 0, 0), 64, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_mm, 64, 0, 0), ks), idn,
                                             ks > 0);
                             tc::mma_commit(s_mbar);
                         }

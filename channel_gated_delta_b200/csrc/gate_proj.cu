@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const uint32_t a = tc::smem_u32(sm + L::STAGES + s * kPStage), bt = a + kPATile;
 #pragma unroll
                 for (int ks = 0; ks < kPK / 16; ++ks)
-                    tc::mma_f16(acc, tc::desc_kmajor(a, kPM, 0, ks), tc::desc_mnmajor(bt, kPK, 0, ks), idesc,
+                    tc::mma_f16(acc, tc::desc_kmajor_step(tc::desc_kmajor(a, kPM, 0, 0), kPM, ks), tc::desc_mnmajor_step(tc::desc_mnmajor(bt, kPK, 0, 0), ks), idesc,
                                 kk > 0 || ks > 0);
                 tc::mma_commit(s_empty + 8 * s);              // the stage is free once these MMAs are done
                 issued = true;

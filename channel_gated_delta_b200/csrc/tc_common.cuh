@@ -60,6 +60,17 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int R, int row0,
     return make_desc(a, (uint32_t)R * 128u, 1024);
 }
 
+// The descriptor of K-step ks from that of step 0: only the start-address field
+// (address >> 4, bits 0-13) moves, and shared-memory addresses stay below 2^18,
+// so a plain add never carries out of the field.  With ks a compile-time
+// constant this is one 64-bit add per MMA instead of rebuilding the descriptor
+// (which, measured, held a single issuing thread to about 100 cycles per MMA
+// against about 70).
+__device__ __forceinline__ uint64_t desc_kmajor_step(uint64_t d0, int R, int ks) {
+    return d0 + (uint64_t)((ks >> 2) * R * 8 + (ks & 3) * 2);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor_step(uint64_t d0, int ks) { return d0 + (uint64_t)(ks * 128); }
+
 // Instruction descriptor, kind::f16 with fp16 A and B, fp32 accumulator.
 __device__ __forceinline__ uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn, bool a_neg) {
     uint32_t d = 0;
