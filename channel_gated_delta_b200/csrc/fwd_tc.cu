@@ -30,6 +30,8 @@
 // which is the unrolled recurrence S_t = Diag(alpha_t)S - k^_t^T(k_t Diag(alpha_t) S)
 // + k_t^T v^_t, o_t = q~_t S_t of the Muir review §2.1 (R holds the erase
 // projections r_t = k_t Diag(alpha_t) S_{t-1}).  y = g * O / rms(O).
+#include <cuda.h>
+#include <cstring>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -1161,12 +1163,21 @@ constexpr uint32_t kItmW = 0;
 constexpr uint32_t kItmN = 16u << 16;
 }  // namespace
 
+// The intra kernel's raw inputs k, q, z, b as 4-D TMA maps over [B, T, H, 128]
+// bf16 (innermost first: channel, head, token, batch; tokens past T read as
+// zeros), boxes of 64 channels x 1 head x 64 tokens x 1 with the 128-byte
+// swizzle: one box is one 64-column block of 64 rows of a row tile.
+struct IntraMaps {
+    CUtensorMap k, q, z, b;
+};
+
 // Input forms, fixed at compile time: kNoZ reads no z (2 sigmoid(z) = 1), kBeta
 // reads one beta per token and head for both b and w, kTok one log-decay per
 // token and head, kRaw applies SiLU and l2 normalisation to q and k.  All false
 // is the per-channel GDN-2 form on preprocessed q and k.
 template <bool kNoZ, bool kBeta, bool kTok, bool kRaw>
-__global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags) {
+__global__ void __launch_bounds__(kThreads, 3)
+    gdn2_chunk_intra_tc_kernel(TcParams p, uint8_t *ws, int *wflags, const __grid_constant__ IntraMaps im) {
     using L = IntraSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1188,6 +1199,7 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
     uint32_t *tslot = (uint32_t *)(sm + L::MISC + 8);
     int *flags = (int *)(sm + L::MISC + 16);
     const uint32_t s_stall = tc::smem_u32(sm + L::MISC + 32);    // never completed (failure-path tests)
+    const uint32_t s_tbar = tc::smem_u32(sm + L::MISC + 40);     // the raw input tiles
     const uint32_t s_ap = tc::smem_u32(sm + L::AP), s_bp = tc::smem_u32(sm + L::BP);
     const uint32_t s_ti = tc::smem_u32(sm + L::TI), s_mm = tc::smem_u32(sm + L::MM);
     const uint32_t s_mbar = tc::smem_u32(mbar);
@@ -1199,11 +1211,26 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
     if (tid == 0) {
         tc::mbar_init(s_mbar, 1);
         tc::mbar_init(s_stall, 1);
+        tc::mbar_init(s_tbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
         // until its record is complete the window is marked for the chain kernel to
         // process itself, so an abandoned record is never read
         wflags[wi] = 1;
+        // The window's raw k, q, z and b, by TMA, straight into the places of the
+        // operand tiles they become (k -> Kp rows, q -> Qp rows of [Kp; Qp]; z -> Kc
+        // rows, b -> K^c rows of [Kc; K^c]): the build turns them over in place, each
+        // thread reading and writing the same elements.  They arrive during the scan.
+        constexpr uint32_t kBox = 64 * 128;                      // one box: 64 rows x 128 bytes
+        tc::mbar_arrive_expect_tx(s_tbar, (uint32_t)((4 - (kNoZ ? 1 : 0) - (kBeta ? 1 : 0)) * 2) * kBox);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t blk = (uint32_t)c * 128 * 128;       // column block c of a 128-row tile
+            tc::tma_load_4d(s_ap + blk, &im.k, 64 * c, h, t0, bb, s_tbar);
+            tc::tma_load_4d(s_ap + blk + kBox, &im.q, 64 * c, h, t0, bb, s_tbar);
+            if (!kNoZ) tc::tma_load_4d(s_bp + blk, &im.z, 64 * c, h, t0, bb, s_tbar);
+            if (!kBeta) tc::tma_load_4d(s_bp + blk + kBox, &im.b, 64 * c, h, t0, bb, s_tbar);
+        }
     }
     if (tid < kDK) gsv[tid] = p.gs ? p.gs[(size_t)h * kDK + tid] : 1.f;
     tc::fence_before_sync();
@@ -1239,8 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
         // factor is one ex2.  Warp w owns tokens [8w, 8w+8), lane l channels [4l, 4l+4)
         // (whole 256-byte token rows per load instruction).  Pass 1 sums the warp's
         // log-decays for the cross-warp prefix; the build below reads them again token
-        // by token (from L2) and keeps only a running sum, so that a thread never holds
-        // more than two tokens' inputs.
+        // by token (from L2, one token ahead) and keeps only a running sum.
         const int tb = 8 * warp, c4 = 4 * lane;
         auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
         auto load_la = [&](int u) -> float4 {
@@ -1255,15 +1281,9 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
             }
             return x;
         };
-        // token u's k, q, z and b (4 bf16 each; zeros past the end of the sequence)
-        auto load_kq = [&](int u, uint2 (&o)[4]) {
-            const bool in = t0 + tb + u < wend;
-            const size_t gt = gt_of(u), gk = gt * kDK + c4;
-            o[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + gk)) : make_uint2(0, 0);
-            o[1] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + gk)) : make_uint2(0, 0);
-            o[2] = in && !kNoZ ? __ldg(reinterpret_cast<const uint2 *>(p.z + gk)) : make_uint2(0, 0);
-            o[3] = !in ? make_uint2(0, 0)
-                  : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.b + gk));
+        // token u's beta, when b comes per token (zeros past the end of the sequence)
+        auto load_beta = [&](int u) -> uint2 {
+            return kBeta && t0 + tb + u < wend ? bf16x4_bcast(p.beta, gt_of(u)) : make_uint2(0, 0);
         };
         float off[4] = {0.f, 0.f, 0.f, 0.f};
         {
@@ -1308,6 +1328,10 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
             }
         }
         const int n = wend - t0;
+        // the raw input tiles, issued at the start
+        if (tid == 0 && !tc::mbar_wait(s_tbar, 0, p.spin)) flags[0] = 1;
+        __syncthreads();
+        if (flags[0] != 0) break;
 
         // ---- operand tiles: P operands to shared memory (Qp, Kc and K^c reach the
         // record from there by bulk copy); the pivot vectors straight to the record
@@ -1329,18 +1353,21 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
             }
             float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
             float4 la_nx = load_la(0);
-            uint2 kq_nx[4];
-            load_kq(0, kq_nx);
+            uint2 beta_nx = load_beta(0);
             float dg[16];                             // [u]: q~.k, [8+u]: q~.(b*k) of token tb+u, this lane's channels
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = tb + u;
                 const bool live = t < n;
                 const float4 la_c = la_nx;
-                const uint2 kq_c[4] = {kq_nx[0], kq_nx[1], kq_nx[2], kq_nx[3]};
-                if (u + 1 < 8) {                      // the next token's inputs are in flight meanwhile
+                const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
+                // this thread's four channels of the raw k, q, z, b (their tile places)
+                const uint2 kq_c[4] = {*(const uint2 *)(sm + L::AP + off_t), *(const uint2 *)(sm + L::AP + off_b),
+                                       kNoZ ? make_uint2(0, 0) : *(const uint2 *)(sm + L::BP + off_t),
+                                       kBeta ? beta_nx : *(const uint2 *)(sm + L::BP + off_b)};
+                if (u + 1 < 8) {                      // the next token's log-decay is in flight meanwhile
                     la_nx = load_la(u + 1);
-                    load_kq(u + 1, kq_nx);
+                    beta_nx = load_beta(u + 1);
                 } else {
                     const bool in = t0 + tb < wend;   // the value side of token 0, for after the build
                     const size_t gt = gt_of(0), gv = gt * kDV + c4;
@@ -1390,7 +1417,6 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
                                                    fmaxf(maxabs(khc, 4), maxabs(qp, 4))));
                 dg[u] = dq;
                 dg[8 + u] = db;
-                const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
                 const uint2 ukp = make_uint2(tc::pack_half2(kp[0], kp[1]), tc::pack_half2(kp[2], kp[3]));
                 const uint2 uqp = make_uint2(tc::pack_half2(qp[0], qp[1]), tc::pack_half2(qp[2], qp[3]));
                 const uint2 ukc = make_uint2(tc::pack_half2(kc[0], kc[1]), tc::pack_half2(kc[2], kc[3]));
@@ -1585,8 +1611,13 @@ __global__ void __launch_bounds__(kThreads, 3) gdn2_chunk_intra_tc_kernel(TcPara
             wflags[wi] = 0;
         }
     } while (false);
-    // the record's bulk copies complete before the CTA's shared memory goes away
-    if (tid == 0) tc::bulk_wait_all();
+    // the record's bulk copies complete before the CTA's shared memory goes away,
+    // and so do the input loads (a window handed to the chain kernel, or an abort,
+    // leaves before waiting for them)
+    if (tid == 0) {
+        tc::bulk_wait_all();
+        tc::mbar_wait(s_tbar, 0, kDrainPolls);
+    }
 
     if (range_max > 60000.f && p.status) atomicCAS(p.status, 0, (int)kDevRange);
     if (flags[0] != 0 && tid == 0 && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
@@ -1605,6 +1636,40 @@ size_t fwd_tc_workspace_bytes(int B, int H, int T) {
 bool fwd_tc_supported(int dtype, int dk, int dv, int chunk) {
     return dtype == GDELTA_BF16 && dk == 128 && dv == 128 && chunk == 64;
 }
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// A [B, T, H, 128] bf16 token tensor as the 4-D map the intra kernel loads from.
+bool input_map(CUtensorMap *m, const void *base, int B, int T, int H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)kDK, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t row = (cuuint64_t)kDK * 2;                  // bytes of one token row of one head
+    const cuuint64_t strides[3] = {row, row * (cuuint64_t)H, row * (cuuint64_t)H * (cuuint64_t)T};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t stream) {
     TcParams p;
@@ -1625,7 +1690,15 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     p.wflags = wflags;
 
     const size_t ismem = (size_t)IntraSmem::TOTAL + 1024;
-    using IntraFn = void (*)(TcParams, uint8_t *, int *);
+    // the raw inputs the intra kernel loads by TMA (z and b only in the forms that read them)
+    IntraMaps im;
+    memset(&im, 0, sizeof(im));
+    if (fp.T > 0) {
+        if (!input_map(&im.k, p.k, fp.B, fp.T, fp.H) || !input_map(&im.q, p.q, fp.B, fp.T, fp.H) ||
+            (p.z && !input_map(&im.z, p.z, fp.B, fp.T, fp.H)) || (p.b && !input_map(&im.b, p.b, fp.B, fp.T, fp.H)))
+            return cudaErrorInvalidValue;
+    }
+    using IntraFn = void (*)(TcParams, uint8_t *, int *, IntraMaps);
 #define GDN2_INTRA_FORMS(R)                                                                                    \
     gdn2_chunk_intra_tc_kernel<false, false, false, R>, gdn2_chunk_intra_tc_kernel<false, false, true, R>,    \
         gdn2_chunk_intra_tc_kernel<false, true, false, R>, gdn2_chunk_intra_tc_kernel<false, true, true, R>,  \
@@ -1637,7 +1710,7 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
                                  (p.decay_tok != 0)];
     cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ismem);
     if (e != cudaSuccess) return e;
-    intra<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags);
+    intra<<<(unsigned)nwin, kThreads, ismem, stream>>>(p, ws, wflags, im);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)ChainSmem::TOTAL + 1024;

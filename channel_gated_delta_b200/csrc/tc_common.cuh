@@ -278,6 +278,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const void *tmap,
         : "memory");
 }
 
+// 4-D tiled TMA load (coordinates innermost first); otherwise as tma_load_2d.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst_smem, const void *tmap, int x, int y, int z, int w,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar)
+        : "memory");
+}
+
 // 2-D tiled TMA store of one box from this CTA's shared memory to the tensor
 // map's global memory (bulk-group completion: bulk_commit, then
 // bulk_wait_read_n / bulk_wait_all).  x, y are the box's first column and row,
