@@ -116,25 +116,50 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
             S[m].w = al * S[m].w - kh * rr.w + kk * vv.w;
         }
     };
-    // token t's key-side and value-side vectors into shared memory (the caller syncs before)
-    auto load_token = [&](int t) {
+    // Token t's inputs for this thread's channel, fetched into registers ahead of
+    // use (two tokens ahead in every pass, so a token's loads are in flight while
+    // the two before it are processed): threads 0-127 the key side of channel
+    // tid (k, log alpha, b, q, z), threads 128-255 the value side of channel
+    // tid - 128 (w, v, dy, g).  The backward step reads the same registers again
+    // instead of reloading.
+    struct Tok {
+        float x0, x1, x2, x3, x4;
+    };
+    const float gs_own = (tid < kBD && p.gs) ? p.gs[(size_t)h * kBD + tid] : 1.f;
+    auto fetch = [&](int t) -> Tok {
+        Tok r{0.f, 0.f, 0.f, 0.f, 0.f};
         const size_t gt = ((size_t)bb * T_ + t) * H + h;
         if (tid < kBD) {
             const size_t gi = gt * kBD + tid;
-            const float kk = ldf(k, gi), al = expf(p.la[gi]);
-            const float gs = p.gs ? p.gs[(size_t)h * kBD + tid] : 1.f;
+            r.x0 = ldf(k, gi);
+            r.x1 = p.la[gi];
+            r.x2 = ldf(b, gi);
+            r.x3 = ldf(q, gi);
+            r.x4 = ldf(z, gi);
+        } else {
+            const size_t gj = gt * kBD + (tid - kBD);
+            r.x0 = ldf(w, gj);
+            r.x1 = ldf(v, gj);
+            r.x2 = p.dy ? p.dy[gj] : 0.f;
+            r.x3 = ldf(g, gj);
+        }
+        return r;
+    };
+    // the token's key-side and value-side vectors into shared memory (the caller
+    // syncs before, so that the previous token's are no longer read, and after)
+    auto stage = [&](const Tok &r) {
+        if (tid < kBD) {
+            const float kk = r.x0, al = expf(r.x1);
             sm.k[tid] = kk;
-            sm.kh[tid] = ldf(b, gi) * kk;
+            sm.kh[tid] = r.x2 * kk;
             sm.ka[tid] = kk * al;
             sm.al[tid] = al;
-            sm.qt[tid] = ldf(q, gi) * gs * two_sigmoid(ldf(z, gi));
+            sm.qt[tid] = r.x3 * gs_own * two_sigmoid(r.x4);
         } else {
             const int j = tid - kBD;
-            const size_t gj = gt * kBD + j;
-            sm.vh[j] = ldf(w, gj) * ldf(v, gj);
-            sm.gdy[j] = p.dy ? ldf(g, gj) * p.dy[gj] : 0.f;
+            sm.vh[j] = r.x0 * r.x1;
+            sm.gdy[j] = r.x3 * r.x2;
         }
-        __syncthreads();
     };
     auto store_rows = [&](float *dst, const float4 (&S)[kBRows]) {
 #pragma unroll
@@ -153,9 +178,13 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
         for (int m = 0; m < kBRows; ++m)
             S[m] = s_in ? ld4(s_in + own + (size_t)8 * m * kBD) : make_float4(0.f, 0.f, 0.f, 0.f);
         store_rows(ckpt, S);
+        Tok c0 = T_ > 0 ? fetch(0) : Tok{}, c1 = T_ > 1 ? fetch(1) : Tok{};
         for (int t = 0; t < T_; ++t) {
             __syncthreads();
-            load_token(t);
+            stage(c0);
+            c0 = c1;
+            if (t + 2 < T_) c1 = fetch(t + 2);
+            __syncthreads();
             fwd_step(S);
             if ((t + 1) % kBC == 0 && (t + 1) / kBC < NC) store_rows(ckpt + (size_t)((t + 1) / kBC) * mat, S);
         }
@@ -176,16 +205,25 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
             float4 S[kBRows];
             load_rows(ckpt + (size_t)c * mat, S);
             store_rows(chunk, S);
+            Tok c0 = fetch(t0), c1 = t0 + 1 < t1 ? fetch(t0 + 1) : Tok{};
             for (int t = t0; t < t1; ++t) {
                 __syncthreads();
-                load_token(t);
+                stage(c0);
+                c0 = c1;
+                if (t + 2 < t1) c1 = fetch(t + 2);
+                __syncthreads();
                 fwd_step(S);
                 store_rows(chunk + (size_t)(t - t0 + 1) * mat, S);
             }
         }
+        Tok n0 = fetch(t1 - 1), n1 = t1 - 2 >= t0 ? fetch(t1 - 2) : Tok{};
         for (int t = t1 - 1; t >= t0; --t) {
             __syncthreads();
-            load_token(t);
+            const Tok cur = n0;                      // token t (also read by steps 2, 4 and 6)
+            stage(cur);
+            n0 = n1;
+            if (t - 2 >= t0) n1 = fetch(t - 2);
+            __syncthreads();
             const float *St = chunk + (size_t)(t - t0 + 1) * mat, *Sp = chunk + (size_t)(t - t0) * mat;
             // (1) o = q~ S_t and r = (k alpha) S_{t-1}: column partials
             {
@@ -237,7 +275,7 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
                 const float rho = sm.scal[0], oo = sm.o[j];
                 sm.dO[j] = rho * sm.gdy[j] - rho * rho * rho / kBD * oo * sm.scal[1];
                 const size_t gj = (((size_t)bb * T_ + t) * H + h) * kBD + j;
-                p.grad_g[gj] = p.dy ? p.dy[gj] * oo * rho : 0.f;
+                p.grad_g[gj] = cur.x2 * oo * rho;
             }
             __syncthreads();
             // (3) dS += q~^T do; dq~ = S_t do^T (rows); k dS and (b*k) dS (columns)
@@ -278,8 +316,8 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
                 }
                 sm.dr[j] = -sb;
                 const size_t gj = (((size_t)bb * T_ + t) * H + h) * kBD + j;
-                p.grad_v[gj] = ldf(w, gj) * sa;
-                p.grad_w[gj] = ldf(v, gj) * sa;
+                p.grad_v[gj] = cur.x0 * sa;
+                p.grad_w[gj] = cur.x1 * sa;
             }
             __syncthreads();
             // (5) row sums dS v^T, -dS r^T, S_{t-1} dr^T, (dS + k^T dr) * S_{t-1}; dS <- Diag(alpha) dS_hat
@@ -316,8 +354,8 @@ __global__ void __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
             if (tid < kBD) {
                 const size_t gi = (((size_t)bb * T_ + t) * H + h) * kBD + tid;
                 const float kk = sm.k[tid], al = sm.al[tid];
-                const float bv = ldf(b, gi), qv = ldf(q, gi), zv = ldf(z, gi);
-                const float gs = p.gs ? p.gs[(size_t)h * kBD + tid] : 1.f;
+                const float bv = cur.x2, qv = cur.x3, zv = cur.x4;
+                const float gs = gs_own;
                 const float ts = two_sigmoid(zv);
                 const float dqt = sm.rows[0][tid], dkh = sm.rows[2][tid];
                 p.grad_k[gi] = sm.rows[1][tid] + al * sm.rows[3][tid] + bv * dkh;
