@@ -621,6 +621,14 @@ def test_backward_matches_autograd_oracle(B, T, H, dtype):
     assert max(e.values()) <= TOL_BWD, e
 
 
+def test_backward_long_sequence_matches_autograd_oracle():
+    """1024 tokens (32 checkpoint chunks) on every head of B2 H4 (the last
+    batch row's last head included), bf16 tokens, a non-zero initial state and
+    state gradient: gradient errors do not grow along the sequence."""
+    e = bwd_errors(*_bwd_case(2, 1024, 4, "bf16", 1024))
+    assert max(e.values()) <= TOL_BWD, e
+
+
 def test_backward_without_tokens_passes_the_state_gradient_through():
     import channel_gated_delta_b200 as gd
     B, H = 1, 2
