@@ -440,9 +440,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             float *ecv = (float *)(buf + L::EV), *fcv = ecv + 128;
             const int wend = min(T, kC * (w + 1));
             const bool fast = loaded_of(B) == w;
-            // tile flag of window w + 2, loaded now and first compared once the window's
-            // products are done, so that its latency is hidden
-            const int wflag2 = (p.ws != nullptr && w + 2 < NW) ? __ldg(p.wflags + wbase + w + 2) : 1;
             // an abort agreed by the readout warps becomes this group's abort at the barrier below
             if (tid == 0 && flags[3] != 0) flags[0] = 1;
             if (fast) {
@@ -562,6 +559,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         tc::mma_commit(s_mbar);
                         tc::mma_commit(s_obar + 8u * slot);      // O of this chunk is final
                     }
+                    // tile flag of window w + 2, loaded while every thread waits for the
+                    // MMAs (loaded at the top of the window, its first use stalled there)
+                    const int wflag2 = (p.ws != nullptr && w + 2 < NW) ? __ldg(p.wflags + wbase + w + 2) : 1;
                     if (wait_mma()) {
                         // the chunk's tiles are free: keep its decay factor; once the window's
                         // last chunk is done, its buffer takes the record of window w + 2
