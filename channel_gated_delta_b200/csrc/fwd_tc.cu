@@ -432,6 +432,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         bool first = true;
         int chunk = 0;
         uint32_t uses0 = 0u, uses1 = 0u;                // chunks that used [R; O] slot 0 / 1
+        // thread 0: a record request held back until the next chunk's first MMA group
+        // is issued, so that the copy's shared-memory writes do not land during the
+        // state rescale
+        int pend_w = -1, pend_b = 0;
         for (int w = 0; w < NW && flags[0] == 0; ++w) {
             const int B = w & 1;
             uint8_t *buf = sm + B * L::BUF, *xbuf = sm + (B ^ 1) * L::BUF;
@@ -448,7 +452,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 infl &= ~(1u << B);
             } else if ((infl >> (B ^ 1)) & 1u) {
                 // the other buffer is this window's scratch: a record arriving there
-                // lands first, and is copied again after the window
+                // lands first (a request still held back is issued now), and is
+                // copied again after the window
+                if (tid == 0 && pend_w >= 0) {
+                    enqueue(pend_w, pend_b);
+                    pend_w = -1;
+                }
                 if (!tc::mbar_wait(s_rbar + 8u * (B ^ 1), (rph >> (B ^ 1)) & 1u, p.spin)) flags[0] = 1;
                 rph ^= 1u << (B ^ 1);
                 infl &= ~(1u << (B ^ 1));
@@ -521,6 +530,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                                             id1, true);
                         }
                         tc::mma_commit(s_mbar);                   // [R; O]: R is read out next
+                        if (pend_w >= 0) {
+                            enqueue(pend_w, pend_b);
+                            pend_w = -1;
+                        }
                         // the state's V^ term runs on the tensor core while R is read out
                         // (the next commit covers it)
                         const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, false);
@@ -569,7 +582,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         main_sync();
                         if (t0 + n == wend) {
                             if (wflag2 == 0) {
-                                if (tid == 0) enqueue(w + 2, B);
+                                if (tid == 0) {
+                                    pend_w = w + 2;
+                                    pend_b = B;
+                                }
                                 set_loaded(B, w + 2);
                                 infl |= 1u << B;
                             } else {
@@ -975,7 +991,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             info[4 * slot + 2] = 1;
             tc::mbar_arrive_local(s_ibar + 8u * slot);
         }
-        if (tid == 0) enqueue(-1, 0);
+        if (tid == 0) {
+            if (pend_w >= 0) enqueue(pend_w, pend_b);   // its buffer is marked in flight: the copy is drained below
+            enqueue(-1, 0);
+        }
         // copies still in flight (the loop ended early) complete before exit
         for (int b = 0; b < 2; ++b)
             if ((infl >> b) & 1u) tc::mbar_wait(s_rbar + 8u * b, (rph >> b) & 1u, kDrainPolls);
