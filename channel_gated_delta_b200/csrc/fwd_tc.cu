@@ -530,10 +530,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                                             id1, true);
                         }
                         tc::mma_commit(s_mbar);                   // [R; O]: R is read out next
-                        if (pend_w >= 0) {
-                            enqueue(pend_w, pend_b);
-                            pend_w = -1;
-                        }
                         // the state's V^ term runs on the tensor core while R is read out
                         // (the next commit covers it)
                         const uint32_t id2 = tc::idesc_f16(128, kDVC, true, true, false);
@@ -542,6 +538,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                             for (int ks = 0; ks < kC / 16; ++ks)
                                 tc::mma_f16(tmem + kTmX, tc::desc_mnmajor_step(tc::desc_mnmajor(s_bp, 128, 0, 0), ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_vh, 64, 0, 0), ks),
                                             id2, true);
+                        // a held-back record request, after this group's last MMA: it
+                        // overlaps the tensor pipe draining
+                        if (pend_w >= 0) {
+                            enqueue(pend_w, pend_b);
+                            pend_w = -1;
+                        }
                     }
                 }
                 if (flags[0] == 0 && wait_mma()) {
