@@ -396,7 +396,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         };
 
         auto win_fast = [&](int w) -> bool { return p.ws != nullptr && w < NW && p.wflags[wbase + w] == 0; };
-        // thread 0: post a record request (window w into buffer b; w < 0 stops the loader)
+        // Thread kAux (warp 2, lane 0; its warp holds no R rows) keeps thread 0, the
+        // MMA issuer, free of everything else: it posts every record request
+        // (window w into buffer b; w < 0 stops the loader) and checks each chunk's
+        // O slot.
+        constexpr int kAux = 64;
         uint32_t nreq = 0;
         auto enqueue = [&](int w, int b) {
             const uint32_t k = nreq++, sl = k & 1u;
@@ -423,7 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         };
         for (int b = 0; b < 2 && flags[0] == 0; ++b)
             if (win_fast(b)) {
-                if (tid == 0) enqueue(b, b);
+                if (tid == kAux) enqueue(b, b);
                 set_loaded(b, b);
                 infl |= 1u << b;
             }
@@ -432,9 +436,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
         bool first = true;
         int chunk = 0;
         uint32_t uses0 = 0u, uses1 = 0u;                // chunks that used [R; O] slot 0 / 1
-        // thread 0: a record request held back until the next chunk's first MMA group
-        // is issued, so that the copy's shared-memory writes do not land during the
-        // state rescale
+        // thread kAux: a record request held back until the next chunk's first MMA
+        // group has completed, so that the copy's shared-memory writes do not land
+        // during the state rescale
         int pend_w = -1, pend_b = 0;
         for (int w = 0; w < NW && flags[0] == 0; ++w) {
             const int B = w & 1;
@@ -454,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                 // the other buffer is this window's scratch: a record arriving there
                 // lands first (a request still held back is issued now), and is
                 // copied again after the window
-                if (tid == 0 && pend_w >= 0) {
+                if (tid == kAux && pend_w >= 0) {
                     enqueue(pend_w, pend_b);
                     pend_w = -1;
                 }
@@ -501,6 +505,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         range_max = fmaxf(range_max, maxabs(v, 32));
                         store_row32(sm + L::SC, 128, i, col, v);
                     }
+                    if (tid == kAux) {
+                        // the slot's previous O has been read out of TMEM (and its chunk
+                        // info); the readout warps learn this chunk's tokens now (to fetch
+                        // the gate early)
+                        const uint32_t us = slot ? uses1 : uses0;
+                        if (us > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (us - 1) & 1u, p.spin))
+                            flags[0] = 1;
+                        info[4 * slot] = t0;
+                        info[4 * slot + 1] = n;
+                        info[4 * slot + 2] = 0;
+                        tc::mbar_arrive_local(s_ibar + 8u * slot);
+                    }
                     first = false;
                     tc::fence_proxy_async();
                     tc::fence_before_sync();
@@ -508,15 +524,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
 
                     // ---- I: [R; O] = [W'; Qp] S_c + [N; Aq] V^ ;  X += Kc^T V^
                     if (tid == 0) {
-                        // the slot's previous O has been read out of TMEM (and its chunk info)
-                        const uint32_t us = slot ? uses1 : uses0;
-                        if (us > 0 && !tc::mbar_wait(s_fbar + 8u * slot, (us - 1) & 1u, p.spin))
-                            flags[0] = 1;
-                        // the readout warps learn the chunk's tokens now (to fetch the gate early)
-                        info[4 * slot] = t0;
-                        info[4 * slot + 1] = n;
-                        info[4 * slot + 2] = 0;
-                        tc::mbar_arrive_local(s_ibar + 8u * slot);
                         tc::fence_after_sync();
                         const uint32_t id1 = tc::idesc_f16(128, kDVC, false, true, false);
                         if (flags[0] == 0) {
@@ -538,15 +545,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                             for (int ks = 0; ks < kC / 16; ++ks)
                                 tc::mma_f16(tmem + kTmX, tc::desc_mnmajor_step(tc::desc_mnmajor(s_bp, 128, 0, 0), ks), tc::desc_mnmajor_step(tc::desc_mnmajor(s_vh, 64, 0, 0), ks),
                                             id2, true);
-                        // a held-back record request, after this group's last MMA: it
-                        // overlaps the tensor pipe draining
-                        if (pend_w >= 0) {
-                            enqueue(pend_w, pend_b);
-                            pend_w = -1;
-                        }
                     }
                 }
                 if (flags[0] == 0 && wait_mma()) {
+                    // a held-back record request (kAux's warp has no R rows below)
+                    if (tid == kAux && pend_w >= 0) {
+                        enqueue(pend_w, pend_b);
+                        pend_w = -1;
+                    }
                     // ---- J: R (rows 0-63) -> fp16 tile
                     if (row < 64) {
                         float v[32];
@@ -584,7 +590,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
                         main_sync();
                         if (t0 + n == wend) {
                             if (wflag2 == 0) {
-                                if (tid == 0) {
+                                if (tid == kAux) {
                                     pend_w = w + 2;
                                     pend_b = B;
                                 }
@@ -979,7 +985,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             // (its scratch buffer) is copied again, and this buffer takes window w + 2
             if (!fast && flags[0] == 0) {
                 if (loaded_of(B ^ 1) == w + 1) {
-                    if (tid == 0) enqueue(w + 1, B ^ 1);
+                    if (tid == kAux) enqueue(w + 1, B ^ 1);
                     infl |= 1u << (B ^ 1);
                 }
             }
@@ -993,7 +999,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
             info[4 * slot + 2] = 1;
             tc::mbar_arrive_local(s_ibar + 8u * slot);
         }
-        if (tid == 0) {
+        if (tid == kAux) {
             if (pend_w >= 0) enqueue(pend_w, pend_b);   // its buffer is marked in flight: the copy is drained below
             enqueue(-1, 0);
         }
