@@ -83,7 +83,7 @@ struct BwdParams {
     const float *dy, *dS_out;
     float eps;
     float *grad_q, *grad_k, *grad_v, *grad_b, *grad_w, *grad_z, *grad_g, *grad_la, *grad_gs, *grad_S_in;
-    float *ws_ckpt, *ws_chunk, *ws_dgam;
+    float *ws_ckpt, *ws_chunk, *ws_dgam, *ws_part;
 };
 
 // Five-gate low-rank projection (gdelta.h, gdelta_gate_proj).

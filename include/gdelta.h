@@ -222,7 +222,11 @@ GDELTA_API gdelta_status gdelta_state_affine(float *S_out, const float *A, const
  * d_v = 128; the pages describe a chunked custom backward (Muir review §2.4,
  * keeping the block inverse and solutions and recomputing boundary decays);
  * this one recomputes states from checkpoints every 32 tokens instead and
- * runs the exact per-token gradient recurrence on CUDA cores.
+ * runs the exact per-token gradient recurrence on CUDA cores, two CTAs per
+ * head (one per half of the value columns).  The key-side gradients
+ * (grad_q, grad_k, grad_z, grad_b, grad_log_alpha) are accumulated from the
+ * two halves: they are zeroed on `stream` first, then written, and must not
+ * alias any input.
  *
  *   B, T, H, dk, dv, dtype, q, k, z, b, v, w, g, log_alpha, gamma_stat,
  *   S_in, eps   : as in gdelta_fwd_args (gamma_stat, S_in may be NULL)
@@ -233,7 +237,9 @@ GDELTA_API gdelta_status gdelta_state_affine(float *S_out, const float *A, const
  *   grad_gamma_stat : [H, d_k] fp32 out (summed over batch and tokens) or NULL
  *   grad_S_in       : [B, H, d_k, d_v] fp32 out or NULL
  *   workspace       : gdelta_bwd_workspace_bytes(args) bytes of device memory
- *                     (checkpoints and one chunk of states per head);
+ *                     (checkpoints and one chunk of states per head and value
+ *                     half, and two RMS partial sums per token, head and
+ *                     warp-pair);
  *                     GDELTA_ERR_WORKSPACE if smaller
  * Unsupported shapes return GDELTA_ERR_UNSUPPORTED.  Asynchronous on `stream`.
  */
