@@ -77,11 +77,10 @@ __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast
 
 struct BwdSmem {
     float k[kBD], kh[kBD], ka[kBD], al[kBD], qt[kBD], qtp[kBD];   // token vectors, key side (qtp: previous token's q~)
-    float vh[kBH], gdy[kBH], gdyp[kBH], o[kBH], r[kBH], dO[kBH], dr[kBH];   // value side, this CTA's columns
+    float vh[kBH], gdy[kBH], gdyp[kBH], r[kBH], dO[kBH], dr[kBH];   // value side, this CTA's columns
     float redA[16][kBH], redB[16][kBH];                      // column partials per (warp, half)
     float rows[5][kBD];                                      // row sums over this CTA's columns
     float2 part[4];                                          // this token's RMS partials (both CTAs)
-    float scal[2];
 };
 
 template <typename T>
@@ -262,14 +261,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
             }
         }
         Tok n0 = fetch(t1 - 1, true), n1 = t1 - 2 >= t0 ? fetch(t1 - 2, true) : Tok{};
+        // this thread's rows of S_t and S_{t-1}, held in registers for the whole
+        // token; walking backward, S_{t-1} of one token is S_t of the next, so each
+        // token loads one state (issued before its barriers)
+        float4 stv[kBRows], spv[kBRows];
+        load_rows(chunk + (size_t)(t1 - t0) * mat, stv);
         for (int t = t1 - 1; t >= t0; --t) {
+            load_rows(chunk + (size_t)(t - t0) * mat, spv);
             __syncthreads();
             const Tok cur = n0;                                // token t (also read by steps 2, 4 and 6)
             stage(cur, false, true);
             n0 = n1;
             if (t - 2 >= t0) n1 = fetch(t - 2, true);
             __syncthreads();
-            const float *St = chunk + (size_t)(t - t0 + 1) * mat, *Sp = chunk + (size_t)(t - t0) * mat;
             const size_t gt = ((size_t)bb * T_ + t) * H + h;
             // (1) o = q~ S_t and r = (k alpha) S_{t-1}: column partials
             {
@@ -277,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
 #pragma unroll
                 for (int m = 0; m < kBRows; ++m) {
                     const int i = row_of(m);
-                    const float4 st = ld4(St + own(m)), sp = ld4(Sp + own(m));
+                    const float4 st = stv[m], sp = spv[m];
                     const float a = sm.qt[i], c2 = sm.ka[i];
                     o4.x = fmaf(a, st.x, o4.x); o4.y = fmaf(a, st.y, o4.y);
                     o4.z = fmaf(a, st.z, o4.z); o4.w = fmaf(a, st.w, o4.w);
@@ -288,28 +292,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                 *reinterpret_cast<float4 *>(&sm.redB[2 * warp + hl][col4]) = r4;
             }
             __syncthreads();
-            if (tid < kBH) {
-                float so = 0.f, sr = 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    so += sm.redA[u][tid];
-                    sr += sm.redB[u][tid];
-                }
-                sm.o[tid] = so;
-                sm.r[tid] = sr;
-            } else if (tid == 64) {
-                // (2a) the RMS norm over both CTAs' columns: the four partial pairs in a fixed order
-                const float *pp = reinterpret_cast<const float *>(sm.part);
-                const float ss = ((pp[0] + pp[2]) + pp[4]) + pp[6], cs = ((pp[1] + pp[3]) + pp[5]) + pp[7];
-                sm.scal[0] = rsqrtf(ss / kBD + p.eps);
-                sm.scal[1] = cs;
-            }
-            __syncthreads();
-            // (2b) do and dg on this CTA's columns
+            // (2) the value side of column j: o and r, the RMS norm over both CTAs'
+            // columns (the four partial pairs, summed in a fixed order), do and dg
             if (tid >= kBD && tid < kBD + kBH) {
                 const int j = tid - kBD;
-                const float rho = sm.scal[0], oo = sm.o[j];
-                sm.dO[j] = rho * sm.gdy[j] - rho * rho * rho / kBD * oo * sm.scal[1];
+                float oo = 0.f, sr = 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    oo += sm.redA[u][j];
+                    sr += sm.redB[u][j];
+                }
+                sm.r[j] = sr;
+                const float *pp = reinterpret_cast<const float *>(sm.part);
+                const float ss = ((pp[0] + pp[2]) + pp[4]) + pp[6], cs = ((pp[1] + pp[3]) + pp[5]) + pp[7];
+                const float rho = rsqrtf(ss / kBD + p.eps);
+                sm.dO[j] = rho * sm.gdy[j] - rho * rho * rho / kBD * oo * cs;
                 p.grad_g[gt * kBD + gc0 + j] = cur.x2 * oo * rho;
             }
             __syncthreads();
@@ -321,7 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
 #pragma unroll
                 for (int m = 0; m < kBRows; ++m) {
                     const int i = row_of(m);
-                    const float4 st = ld4(St + own(m));
+                    const float4 st = stv[m];
                     rowv[m] = dot4(st, d4);
                     float4 ds = sdS[i * 16 + lc];
                     const float a = sm.qt[i];
@@ -362,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
 #pragma unroll
                 for (int m = 0; m < kBRows; ++m) {
                     const int i = row_of(m);
-                    const float4 sp = ld4(Sp + own(m));
+                    const float4 sp = spv[m];
                     float4 ds = sdS[i * 16 + lc];
                     ra[m] = dot4(ds, vv);
                     rb[m] = -dot4(ds, rr);
@@ -399,6 +396,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                 atomicAdd(p.grad_z + gi, dqt * qv * gs_own * ts * (1.f - 0.5f * ts));
                 dgam = fmaf(dqt * qv, ts, dgam);
             }
+#pragma unroll
+            for (int m = 0; m < kBRows; ++m) stv[m] = spv[m];
         }
     }
     __syncthreads();
