@@ -646,7 +646,7 @@ def run_bwd(args, gd, d, shape, dev, stream, world):
             "tokens_per_s": B * T * world / (ms * 1e-3), "algorithmic_bytes": nb,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
             "timed_calls": args.bwd_calls,
-            "note": f"one CTA per head walks its tokens in order: latency-bound, {B * H} CTAs"}
+            "note": f"a two-CTA cluster per head (value halves) walks the tokens in order: latency-bound, {2 * B * H} CTAs"}
 
 
 def run_stream(args, gd, d, shape, dev, stream, world, decode_steps=256):
