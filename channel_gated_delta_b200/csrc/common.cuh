@@ -92,7 +92,7 @@ struct GateProjParams {
     int ranks[5];
     const void *x, *w_down, *w_up;
     const float *bias;
-    void *codes;             // workspace: [N, R] bf16
+    void *codes;             // workspace: [N, 2R] bf16, the codes as two parts (hi | lo)
     float *log_alpha;
     void *b, *g, *w, *z;
     int *status;
