@@ -41,8 +41,13 @@ constexpr int kPK = 64;                           // contraction per stage (128 
 constexpr int kPATile = kPM * kPK * 2;            // 16 KiB
 constexpr int kPBTile = kPK * kPN * 2;            // 32 KiB: 4 column blocks of 64 x 64
 constexpr int kPStage = kPATile + kPBTile;
-constexpr int kPThreads = 320;                   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-constexpr int kPEpiWarps = 8;
+// warp 0 TMA, warp 1 MMA, then the epilogue warps: 8 for down (two per TMEM lane
+// quadrant, 128 columns each), 16 for up (four per quadrant, 64 columns each:
+// its epilogue, with the bias and the activations, is what bounds it)
+template <bool kUp>
+constexpr int epi_warps() { return kUp ? 16 : 8; }
+template <bool kUp>
+constexpr int proj_threads() { return 64 + 32 * epi_warps<kUp>(); }
 constexpr int kPBox = 32 * 128;                   // one staged output box: 32 rows of 128 bytes
 constexpr uint32_t kPDrainPolls = 1u << 22;
 
@@ -54,8 +59,8 @@ struct ProjSmem {
     static constexpr int kStages = kUp ? 3 : 4;
     static constexpr int STAGES = 0;
     static constexpr int OUT = kStages * kPStage;
-    static constexpr int BIAS = OUT + (kUp ? kPEpiWarps * 2 * kPBox : 0);
-    static constexpr int BAR = BIAS + (kUp ? kPEpiWarps * 128 * 4 : 0);  // full, empty, acc_full[2], acc_empty[2], stall
+    static constexpr int BIAS = OUT + (kUp ? epi_warps<kUp>() * kPBox : 0);        // one staged box per warp
+    static constexpr int BAR = BIAS + (kUp ? epi_warps<kUp>() * 64 * 4 : 0);    // full, empty, acc_full[2], acc_empty[2], stall
     static constexpr int MISC = BAR + 8 * (2 * kStages + 5);              // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 64;
     static_assert(OUT % 1024 == 0, "staged boxes start on a 1024-byte boundary");
@@ -144,7 +149,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 }  // namespace
 
 template <bool kUp>
-__global__ void __launch_bounds__(kPThreads, 1)
+__global__ void __launch_bounds__(proj_threads<kUp>(), 1)
     gate_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const __grid_constant__ ProjParams p) {
     using L = ProjSmem<kUp>;
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(s_accf + 8 * b, 1);
-            tc::mbar_init(s_acce + 8 * b, kPEpiWarps);
+            tc::mbar_init(s_acce + 8 * b, epi_warps<kUp>());
         }
         tc::mbar_init(s_stall, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -300,24 +305,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (timed_out && lane == 0) *abort_flag = 1;
     } else if (warp >= 2) {
         // ---- up epilogue.  The warp owns TMEM lanes 32 (warp % 4) .. +31 (the
-        // tile's rows) and 128 of its columns (warps 2-5 the first half, 6-9 the
-        // second).  Activated values are staged in shared memory as boxes of 32
-        // rows x 128 bytes (32 fp32 or 64 bf16 columns), each row's 16-byte chunks
-        // in the 128-byte-swizzled order (chunk q at q ^ (row % 8): the eight rows
-        // a store phase covers hit eight different bank groups), and lane 0 writes
-        // each box with one TMA store (one bulk group per box); the warp's two
-        // box buffers alternate.
-        const int ew = warp - 2, qd = warp & 3, cbase = warp < 6 ? 0 : kPN / 2;
-        const uint32_t obuf = tc::smem_u32(sm + L::OUT + ew * 2 * kPBox);
-        float *sbias = reinterpret_cast<float *>(sm + L::BIAS + ew * 128 * 4);
+        // tile's rows) and 64 of its columns (warps 2-5 the first quarter, 6-9 the
+        // second, ...).  Activated values are staged in shared memory as boxes of
+        // 32 rows x 128 bytes (32 fp32 or 64 bf16 columns), each row's 16-byte
+        // chunks in the 128-byte-swizzled order (chunk q at q ^ (row % 8): the
+        // eight rows a store phase covers hit eight different bank groups), and
+        // lane 0 writes each box with one TMA store; the warp's one box buffer is
+        // refilled once the previous store has read it.
+        const int ew = warp - 2, qd = warp & 3, cbase = 64 * (ew >> 2);
+        const uint32_t obuf = tc::smem_u32(sm + L::OUT + ew * kPBox);
+        float *sbias = reinterpret_cast<float *>(sm + L::BIAS + ew * 64 * 4);
         const uint32_t rowoff = (uint32_t)lane * 128u, sw = (uint32_t)(lane & 7);
-        uint32_t t = 0, nbox = 0;
+        uint32_t t = 0;
         for (int j = blockIdx.x; j < p.jobs; j += gridDim.x, ++t) {
             const Job jb = job_of<kUp>(p, j);
             const uint32_t b = t & 1u, v = t >> 1;
-            // this warp's 128 bias values, fetched before the accumulator wait
-            const float4 bv =
-                __ldg(reinterpret_cast<const float4 *>(p.bias + (size_t)jb.gate * p.d + jb.n0 + cbase) + lane);
+            // this warp's 64 bias values, fetched before the accumulator wait
+            const float4 bv = lane < 16 ? __ldg(reinterpret_cast<const float4 *>(p.bias + (size_t)jb.gate * p.d +
+                                                                                 jb.n0 + cbase) + lane)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
             bool ok = true;
             if (lane == 0) ok = !*abort_flag && tc::mbar_wait(s_accf + 8 * b, v & 1u, p.spin);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -337,88 +343,64 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 release();
                 continue;
             }
-            reinterpret_cast<float4 *>(sbias)[lane] = bv;
+            if (lane < 16) reinterpret_cast<float4 *>(sbias)[lane] = bv;
             __syncwarp();
             const CUtensorMap *map = jb.gate == 0 ? &om.la : jb.gate == 1 ? &om.gb : jb.gate == 2 ? &om.gg
                                      : jb.gate == 3 ? &om.gw : &om.gz;
-            // two rounds of 64 columns: both TMEM loads of a round, then one wait;
-            // the log-decay (fp32) fills two boxes of 32 columns per round, the
-            // bf16 gates one box of 64
-            const int x0 = jb.n0 + cbase;
 #pragma unroll 1
-            for (int r = 0; r < 2; ++r) {
-                float va[32], vb[32];
-                tc::tmem_ld32x2(acc + 64 * r, acc + 64 * r + 32, va, vb);
-                if (r == 1) release();
-                const float4 *bb = reinterpret_cast<const float4 *>(sbias + 64 * r);
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[32];
+                tc::tmem_ld32(acc + 32 * hh, x);
+                if (hh == 1) release();
+                const float4 *bb = reinterpret_cast<const float4 *>(sbias + 32 * hh);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 c4 = bb[q], d4 = bb[8 + q];
-                    va[4 * q] += c4.x; va[4 * q + 1] += c4.y; va[4 * q + 2] += c4.z; va[4 * q + 3] += c4.w;
-                    vb[4 * q] += d4.x; vb[4 * q + 1] += d4.y; vb[4 * q + 2] += d4.z; vb[4 * q + 3] += d4.w;
+                    const float4 c4 = bb[q];
+                    x[4 * q] += c4.x; x[4 * q + 1] += c4.y; x[4 * q + 2] += c4.z; x[4 * q + 3] += c4.w;
                 }
                 if (jb.gate == 0) {
+                    // log alpha: a box of 32 fp32 columns per half
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        va[i] = plogsigmoid(va[i]);
-                        vb[i] = plogsigmoid(vb[i]);
-                    }
-                    // both buffers: the stores issued before have finished reading them
+                    for (int i = 0; i < 32; ++i) x[i] = plogsigmoid(x[i]);
                     if (lane == 0) tc::bulk_wait_read_n<0>();
                     __syncwarp();
-                    const uint32_t ba = obuf + (nbox & 1u) * kPBox, bq = obuf + ((nbox + 1) & 1u) * kPBox;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        st_shared_v4(ba + rowoff + ((q ^ sw) << 4), __float_as_uint(va[4 * q]),
-                                     __float_as_uint(va[4 * q + 1]), __float_as_uint(va[4 * q + 2]),
-                                     __float_as_uint(va[4 * q + 3]));
-                        st_shared_v4(bq + rowoff + ((q ^ sw) << 4), __float_as_uint(vb[4 * q]),
-                                     __float_as_uint(vb[4 * q + 1]), __float_as_uint(vb[4 * q + 2]),
-                                     __float_as_uint(vb[4 * q + 3]));
-                    }
+                    for (int q = 0; q < 8; ++q)
+                        st_shared_v4(obuf + rowoff + (((uint32_t)q ^ sw) << 4), __float_as_uint(x[4 * q]),
+                                     __float_as_uint(x[4 * q + 1]), __float_as_uint(x[4 * q + 2]),
+                                     __float_as_uint(x[4 * q + 3]));
                     tc::fence_proxy_async();
                     __syncwarp();
                     if (lane == 0) {
-                        tc::tma_store_2d(map, ba, x0 + 64 * r, y);
-                        tc::bulk_commit();
-                        tc::tma_store_2d(map, bq, x0 + 64 * r + 32, y);
+                        tc::tma_store_2d(map, obuf, jb.n0 + cbase + 32 * hh, y);
                         tc::bulk_commit();
                     }
-                    nbox += 2;
                 } else {
+                    // a bf16 gate: both halves fill one box of 64 columns (chunks 4 hh .. 4 hh + 3)
                     if (jb.gate == 1) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            va[i] = 2.f * psigmoid(va[i]);
-                            vb[i] = 2.f * psigmoid(vb[i]);
-                        }
+                        for (int i = 0; i < 32; ++i) x[i] = 2.f * psigmoid(x[i]);
                     } else if (jb.gate != 4) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            va[i] = psigmoid(va[i]);
-                            vb[i] = psigmoid(vb[i]);
+                        for (int i = 0; i < 32; ++i) x[i] = psigmoid(x[i]);
+                    }
+                    if (hh == 0) {
+                        if (lane == 0) tc::bulk_wait_read_n<0>();
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(obuf + rowoff + (((uint32_t)(4 * hh + q) ^ sw) << 4), pack_bf2(x[8 * q], x[8 * q + 1]),
+                                     pack_bf2(x[8 * q + 2], x[8 * q + 3]), pack_bf2(x[8 * q + 4], x[8 * q + 5]),
+                                     pack_bf2(x[8 * q + 6], x[8 * q + 7]));
+                    if (hh == 1) {
+                        tc::fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tc::tma_store_2d(map, obuf, jb.n0 + cbase, y);
+                            tc::bulk_commit();
                         }
                     }
-                    // this buffer was last read by the store two boxes back
-                    if (lane == 0) tc::bulk_wait_read_n<1>();
-                    __syncwarp();
-                    const uint32_t ba = obuf + (nbox & 1u) * kPBox;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        st_shared_v4(ba + rowoff + (((uint32_t)q ^ sw) << 4), pack_bf2(va[8 * q], va[8 * q + 1]),
-                                     pack_bf2(va[8 * q + 2], va[8 * q + 3]), pack_bf2(va[8 * q + 4], va[8 * q + 5]),
-                                     pack_bf2(va[8 * q + 6], va[8 * q + 7]));
-                        st_shared_v4(ba + rowoff + (((uint32_t)(4 + q) ^ sw) << 4), pack_bf2(vb[8 * q], vb[8 * q + 1]),
-                                     pack_bf2(vb[8 * q + 2], vb[8 * q + 3]), pack_bf2(vb[8 * q + 4], vb[8 * q + 5]),
-                                     pack_bf2(vb[8 * q + 6], vb[8 * q + 7]));
-                    }
-                    tc::fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tc::tma_store_2d(map, ba, x0 + 64 * r, y);
-                        tc::bulk_commit();
-                    }
-                    nbox += 1;
                 }
             }
         }
@@ -528,7 +510,7 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     p.nn = p.R / kPN;
     p.jobs = mt * p.nn;
-    gate_proj_kernel<false><<<min(sms[dev], p.jobs), kPThreads, smem_down, stream>>>(ta, tb, om, p);
+    gate_proj_kernel<false><<<min(sms[dev], p.jobs), proj_threads<false>(), smem_down, stream>>>(ta, tb, om, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // up: A = codes [N, 2R] (hi | lo), B = w_up [R, d]; the five outputs
@@ -540,7 +522,7 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     p.nn = gp.d / kPN;
     p.jobs = mt * 5 * p.nn;
-    gate_proj_kernel<true><<<min(sms[dev], p.jobs), kPThreads, smem_up, stream>>>(ta, tb, om, p);
+    gate_proj_kernel<true><<<min(sms[dev], p.jobs), proj_threads<true>(), smem_up, stream>>>(ta, tb, om, p);
     return cudaGetLastError();
 }
 
