@@ -553,9 +553,56 @@ def run_configs(args, gd, dev, stream, rank, world):
                          "peak_source": kind, "algorithmic_bytes_per_launch": nb, "launch_ms": ms},
             "l2": "inputs larger than the 126 MB L2; no flush",
         }
+        if B == 1 and T >= 16384 and T % (4 * C) == 0:
+            out[name]["segment_scan"] = run_segment_scan(gd, d, shape, y, dev, stream, world, args, 4)
         del d, S, y, ws
         torch.cuda.empty_cache()
     return out
+
+
+def run_segment_scan(gd, d, shape, y_direct, dev, stream, world, args, P):
+    """One sequence (B = 1) as P segments on one GPU: the segments' affine state
+    maps (gdelta_segment_map: two forward calls over the P segments as batch
+    rows), their composition into each segment's starting state
+    (gdelta_state_affine), and the forward over the segments from those states.
+    Timed against the direct call above; y compared with it."""
+    T, H, dk, dv, C = shape.T, shape.H, shape.dk, shape.dv, shape.chunk
+    Ts = T // P
+    seg = {k: d[k].view(P, Ts, *d[k].shape[2:]) for k in ("q", "k", "v", "b", "w", "z", "g", "log_alpha")}
+    S_start = torch.zeros(P, H, dk, dv, device=dev)
+    S_end = torch.empty(P, H, dk, dv, device=dev)
+    ys = torch.empty(P, Ts, H, dv, dtype=torch.bfloat16, device=dev)
+
+    def call():
+        A, D = gd.gdelta_segment_map(seg["q"], seg["k"], seg["v"], seg["b"], seg["w"], seg["z"], seg["g"],
+                                     seg["log_alpha"], chunk=C, path=args.path, stream=stream)
+        for j in range(1, P):
+            gd.gdelta_state_affine(A[j - 1:j], S_start[j - 1:j], D[j - 1:j], S_out=S_start[j:j + 1], stream=stream)
+        gd.gdelta_fwd_chunked(seg["q"], seg["k"], seg["v"], seg["b"], seg["w"], seg["z"], seg["g"],
+                              seg["log_alpha"], gamma_stat=d["gamma_stat"], S_in=S_start, S_out=S_end, y=ys,
+                              chunk=C, path=args.path, stream=stream)
+
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize(dev)
+    if gd.gdelta_get_last_device_error(stream) != 0:
+        raise RuntimeError("device status word set during the segment scan")
+    n = max(3, min(args.steps, 5))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier(world)
+    for a, c in evs:
+        a.record(stream)
+        call()
+        c.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(statistics.median(a.elapsed_time(c) for a, c in evs), world)
+    ref = y_direct.float().view(-1)
+    diff = float((ys.float().view(-1) - ref).abs().max() / ref.pow(2).mean().sqrt())
+    return {"segments": P, "ms_median": ms, "tokens_per_s": T * world / (ms * 1e-3),
+            "y_max_abs_diff_over_rms_vs_direct": diff,
+            "note": "three forward calls over T/P tokens in P rows (the map's two, then the final one) "
+                    "against the direct call's one over T: on one GPU the chain already has 128 CTAs' "
+                    "worth of work at P = 4"}
 
 
 def run_gate_proj(args, gd, shape, dev, stream, rank, world):
