@@ -13,13 +13,20 @@
 //      one cluster barrier after phase F, and every later read sums the four
 //      pairs in the same order, so both CTAs use the same rho;
 //  (b) each CTA adds its share of dk, db, d log alpha, dq, dz to the outputs
-//      (zeroed by the launcher) with atomics: two addends to a zero, so the
-//      result does not depend on their order.
+//      (zeroed by the launcher) with atomic reductions: two addends to a zero,
+//      so the result does not depend on their order.
 //
 // Phase F runs the recurrence forward and keeps the state every kBC tokens
-// (checkpoints).  Phase B walks the chunks from the last: it recomputes the
-// chunk's kBC + 1 states from its checkpoint into a per-CTA buffer, then takes
-// the tokens in reverse with the exact per-token gradient recurrence below.
+// (checkpoints), and each token's o and r on this CTA's columns.  Phase B walks
+// the chunks from the last: it recomputes the chunk's kBC + 1 states from its
+// checkpoint (with the stored r, a state step needs no column sum and one
+// barrier a token), passing them through two shared-memory tiles to a per-CTA
+// chunk buffer by bulk copies, then takes the tokens in reverse with the exact
+// per-token gradient recurrence below (o and r again from phase F), loading
+// each state back by bulk copy one token ahead.  Per-token inputs are fetched
+// into registers a few tokens ahead (phase F and the recompute: four, the
+// walk: two), the token loops unrolled so that the register sets rotate
+// without moves.
 // Per token, with S_hat = Diag(alpha) S_{t-1}, r = k S_hat,
 // S_t = S_hat - (b*k)^T r + k^T (w*v), o = q~ S_t and y = g * o * rho,
 // rho = 1 / sqrt(mean(o^2) + eps) (Muir review §2.1):
@@ -31,9 +38,9 @@
 //   dS_hat  = dS + k^T dr     dalpha = rowsum(dS_hat * S_{t-1}) dS_{t-1} = Diag(alpha) dS_hat
 //
 // and the chain rule through q~ = q * gamma * 2 sigmoid(z), v^ = w * v,
-// alpha = exp(log_alpha).  The checkpoints, chunk states and RMS partials live
-// in the caller's workspace; the running dS (this CTA's half) lives in shared
-// memory.
+// alpha = exp(log_alpha).  The checkpoints, chunk states, per-token o and r and
+// RMS partials live in the caller's workspace; the running dS (this CTA's half)
+// lives in shared memory.
 //
 // Thread layout (256 threads): warp w, lane l = 16 h + c holds rows
 // w + 8 h + 16 m (m = 0..7) and the CTA's columns 4c..4c+3, so a row's sum over
@@ -51,6 +58,11 @@ constexpr int kBH = 64;              // value columns per CTA
 constexpr int kBT = 256;             // threads
 constexpr int kBRows = 8;            // rows per thread
 constexpr int kBC = 32;              // tokens per checkpoint
+constexpr uint32_t kSlotBytes = kBD * kBH * 4;   // one [128][64] fp32 state half-matrix
+constexpr uint32_t kBwdDrainPolls = 1u << 22;    // polls of the wait that drains a copy after a timeout
+// The thread that issues the walk's state loads: in warp 6, which has no key or
+// value role, so that its proxy fence never waits on gradient atomics.
+constexpr int kLoader = 192;
 
 // Reduce-scatter of 8 per-lane values over a half-warp: afterwards lane l
 // holds the sum over its 16 lanes of value (l >> 1) & 7.
@@ -72,16 +84,47 @@ __device__ __forceinline__ float rows_reduce_scatter8(const float (&v)[8], int l
     return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
 }
 
+// An input element's raw bits, converted to fp32 only where it is used: a value
+// fetched tokens ahead of its use then keeps its load in flight instead of
+// stalling the warp at the conversion right after the load.
+__device__ __forceinline__ uint32_t ldraw(const float *p, size_t i) { return __float_as_uint(p[i]); }
+__device__ __forceinline__ uint32_t ldraw(const __nv_bfloat16 *p, size_t i) {
+    return (uint32_t)reinterpret_cast<const unsigned short *>(p)[i];
+}
+__device__ __forceinline__ float cvraw(uint32_t x, const float *) { return __uint_as_float(x); }
+__device__ __forceinline__ float cvraw(uint32_t x, const __nv_bfloat16 *) { return __uint_as_float(x << 16); }
+
+// Atomic add with no return value (a reduction): the issuing thread never waits
+// for the old value to come back from L2.
+__device__ __forceinline__ void red_add(float *p, float x) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
+}
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 
-struct BwdSmem {
-    float k[kBD], kh[kBD], ka[kBD], al[kBD], qt[kBD], qtp[kBD];   // token vectors, key side (qtp: previous token's q~)
-    float vh[kBH], gdy[kBH], gdyp[kBH], r[kBH], dO[kBH], dr[kBH];   // value side, this CTA's columns
-    float redA[16][kBH], redB[16][kBH];                      // column partials per (warp, half)
-    float rows[5][kBD];                                      // row sums over this CTA's columns
-    float2 part[4];                                          // this token's RMS partials (both CTAs)
+// One token's vectors in shared memory.  Two of these alternate by token
+// parity, so that staging a token never overwrites what the previous one is
+// still being read from; the barriers each phase needs for its own data order
+// the rest.
+struct __align__(16) TokBuf {
+    float k[kBD], kh[kBD], ka[kBD], al[kBD], qt[kBD];        // key side: k, b*k, k*alpha, alpha, q~
+    float vh[kBH], r[kBH], dO[kBH];                           // value side, this CTA's columns: w*v, r, do
 };
+
+struct BwdSmem {
+    TokBuf tb[2];
+    float dr[kBH];                                            // dr of the token being walked
+    float redA[16][kBH], redB[16][kBH];                       // column partials per (warp, half)
+    float rows[5][kBD];                                       // row sums over this CTA's columns
+};
+
+// fmaf form of S_t = alpha S_{t-1} - (b*k) r + k (w*v) for one element, shared by
+// phase F and the recompute so that the recomputed states equal the checkpointed
+// trajectory bit for bit
+__device__ __forceinline__ float state_step(float s, float al, float kh, float rj, float kk, float vj) {
+    return fmaf(kk, vj, fmaf(-kh, rj, al * s));
+}
 
 template <typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
@@ -98,59 +141,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     float *ckpt = p.ws_ckpt + hc * (NC + 1) * mat;
     float *chunk = p.ws_chunk + hc * (kBC + 1) * mat;
     float *part = p.ws_part + (size_t)head * T_ * 8;         // per token: (sum o^2, sum g dy o) x 4 warps-of-a-CTA
+    float *orw = p.ws_or + hc * (size_t)T_ * 2 * kBH;        // per token: o, then r, of this CTA's columns
     const T *q = (const T *)p.q, *k = (const T *)p.k, *z = (const T *)p.z, *b = (const T *)p.b;
     const T *v = (const T *)p.v, *w = (const T *)p.w, *g = (const T *)p.g;
+    const bool keyt = tid < kBD, valt = tid >= kBD && tid < kBD + kBH;
+    const int j = tid - kBD;                                  // a value thread's column in this CTA
     auto row_of = [&](int m) { return warp + 8 * hl + 16 * m; };
     auto own = [&](int m) { return (size_t)row_of(m) * kBH + col4; };           // in a half-matrix buffer
     auto own_full = [&](int m) { return (size_t)row_of(m) * kBD + gc0 + col4; };  // in a [128][128] matrix
-
-    // Token t's inputs for this thread, fetched into registers two tokens ahead
-    // of use: threads 0-127 the key side of channel tid (k, log alpha, b, q, z),
-    // threads 128-191 the value side of this CTA's column tid - 128 (w, v, dy,
-    // g), and in phase B threads 0-7 the token's eight RMS partials.  The
-    // gradient step reads the same registers again instead of reloading.
-    struct Tok {
-        float x0, x1, x2, x3, x4, x5;
+    // Two state tiles in shared memory (each a [128][64] half-matrix, the chunk
+    // buffer's layout) and their mbarriers, after the running dS.  The chunk's
+    // states move between them and the chunk buffer by bulk copies (one thread,
+    // 32 KiB each), which keeps that traffic off the threads' load/store path.
+    float *const slot0 = reinterpret_cast<float *>(sdS + kBD * 16);
+    auto slot = [&](int x) { return slot0 + (size_t)x * mat; };
+    const uint32_t s_slot0 = tc::smem_u32(slot0), s_mb = s_slot0 + 2 * kSlotBytes;
+    uint32_t ph = 0;                                          // bit x: parity of the next wait on slot x
+    if (tid == 0) {
+        tc::mbar_init(s_mb, 1);
+        tc::mbar_init(s_mb + 8, 1);
+    }
+    __syncthreads();
+    // bounded wait for slot x's bulk load; a wait that runs out is reported and then
+    // drained, so that no copy is still landing when the slot is used again
+    auto wait_slot = [&](int x) {
+        const uint32_t mb = s_mb + 8 * x, par = (ph >> x) & 1u;
+        if (!tc::mbar_wait(mb, par, p.wait_limit)) {
+            if (p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
+            tc::mbar_wait(mb, par, kBwdDrainPolls);
+        }
+        ph ^= 1u << x;
     };
-    const float gs_own = (tid < kBD && p.gs) ? p.gs[(size_t)h * kBD + tid] : 1.f;
-    auto fetch = [&](int t, bool with_part) -> Tok {
-        Tok r{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+
+    // Token t's inputs, fetched into registers tokens ahead of use (raw bits; cv
+    // and fl convert them): the key side of channel tid & 127 (k0-k4: k, log
+    // alpha, b, q, z), used by threads 0-127, and the value side of this CTA's
+    // column tid & 63 (v0-v5: w, v, dy, g, and in phase B r and o; in the walk
+    // also the token's eight RMS partials), used by threads 128-191.  Every thread
+    // loads every field, from an index that is valid for any thread: a field that
+    // one role loads and another leaves alone would make the compiler merge the
+    // two at the end of the branch, and that merge waits for the load.  The
+    // gradient step reads the same registers again.  Phases: kF (forward,
+    // checkpoints), kRe (recompute a chunk), kWalk.
+    enum { kF = 0, kRe = 1, kWalk = 2 };
+    struct Tok {
+        uint32_t k0, k1, k2, k3, k4;
+        uint32_t v0, v1, v2, v3, v4, v5;
+        float4 pa, pb;
+    };
+    auto cv = [&](uint32_t x) { return cvraw(x, q); };       // a token-dtype input
+    auto fl = [](uint32_t x) { return __uint_as_float(x); };  // an fp32 input
+    const float gs_own = (keyt && p.gs) ? p.gs[(size_t)h * kBD + tid] : 1.f;
+    const float *dy_src = p.dy ? p.dy : p.la;                  // (read but unused when dy is absent)
+    auto fetch = [&](int t, int ph) -> Tok {
+        Tok r;
         const size_t gt = ((size_t)bb * T_ + t) * H + h;
-        if (tid < kBD) {
-            const size_t gi = gt * kBD + tid;
-            r.x0 = ldf(k, gi);
-            r.x1 = p.la[gi];
-            r.x2 = ldf(b, gi);
-            r.x3 = ldf(q, gi);
-            r.x4 = ldf(z, gi);
-            if (with_part && tid < 8) r.x5 = part[(size_t)t * 8 + tid];
-        } else if (tid < kBD + kBH) {
-            const size_t gj = gt * kBD + gc0 + (tid - kBD);
-            r.x0 = ldf(w, gj);
-            r.x1 = ldf(v, gj);
-            r.x2 = p.dy ? p.dy[gj] : 0.f;
-            r.x3 = ldf(g, gj);
+        const size_t gi = gt * kBD + (tid & (kBD - 1)), gj = gt * kBD + gc0 + (tid & (kBH - 1));
+        const size_t oj = (size_t)t * 2 * kBH + (tid & (kBH - 1));
+        r.k0 = ldraw(k, gi);
+        r.k1 = ldraw(p.la, gi);
+        r.k2 = ldraw(b, gi);
+        r.v0 = ldraw(w, gj);
+        r.v1 = ldraw(v, gj);
+        if (ph != kRe) {
+            r.k3 = ldraw(q, gi);
+            r.k4 = ldraw(z, gi);
+            r.v2 = ldraw(dy_src, gj);
+            r.v3 = ldraw(g, gj);
+        }
+        if (ph != kF) r.v4 = ldraw(orw, oj + kBH);
+        if (ph == kWalk) {
+            r.v5 = ldraw(orw, oj);
+            r.pa = ld4(part + (size_t)t * 8);
+            r.pb = ld4(part + (size_t)t * 8 + 4);
         }
         return r;
     };
-    // the token's vectors into shared memory (the caller syncs before and after);
-    // keep_prev: first move this token's predecessor's q~ and g*dy aside (phase F
-    // reduces o of the previous token with the next token's r)
-    auto stage = [&](const Tok &r, bool keep_prev, bool with_part) {
-        if (tid < kBD) {
-            if (keep_prev) sm.qtp[tid] = sm.qt[tid];
-            const float kk = r.x0, al = expf(r.x1);
-            sm.k[tid] = kk;
-            sm.kh[tid] = r.x2 * kk;
-            sm.ka[tid] = kk * al;
-            sm.al[tid] = al;
-            sm.qt[tid] = r.x3 * gs_own * two_sigmoid(r.x4);
-            if (with_part && tid < 8) reinterpret_cast<float *>(sm.part)[tid] = r.x5;
-        } else if (tid < kBD + kBH) {
-            const int j = tid - kBD;
-            if (keep_prev) sm.gdyp[j] = sm.gdy[j];
-            sm.vh[j] = r.x0 * r.x1;
-            sm.gdy[j] = r.x3 * r.x2;
+    auto dy_of = [&](const Tok &r) { return p.dy ? fl(r.v2) : 0.f; };
+    // the token's vectors into buffer bf (no barrier here: see TokBuf)
+    auto stage = [&](const Tok &r, int ph, TokBuf &bf) {
+        if (keyt) {
+            const float kk = cv(r.k0), al = expf(fl(r.k1));
+            bf.k[tid] = kk;
+            bf.kh[tid] = cv(r.k2) * kk;
+            bf.al[tid] = al;
+            if (ph == kF) bf.ka[tid] = kk * al;
+            if (ph != kRe) bf.qt[tid] = cv(r.k3) * gs_own * two_sigmoid(cv(r.k4));
+        } else if (valt) {
+            bf.vh[j] = cv(r.v0) * cv(r.v1);
+            if (ph != kF) bf.r[j] = fl(r.v4);
         }
     };
     auto store_rows = [&](float *dst, const float4 (&S)[kBRows]) {
@@ -161,77 +240,114 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
 #pragma unroll
         for (int m = 0; m < kBRows; ++m) S[m] = ld4(src + own(m));
     };
-    // r = (k alpha) S (column sums over the rows) and, when o_tok >= 0, o of the
-    // previous token, q~_prev S, whose RMS partials go to the workspace; then,
-    // when update, the state step of the staged token
-    auto fwd_step = [&](float4 (&S)[kBRows], int o_tok, bool update) {
-        float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f), o4 = r4;
+    // S <- S_t of the staged token, given its r on this thread's columns
+    auto update = [&](float4 (&S)[kBRows], const TokBuf &bf, float4 rr) {
+        const float4 vv = ld4(&bf.vh[col4]);
 #pragma unroll
         for (int m = 0; m < kBRows; ++m) {
             const int i = row_of(m);
-            const float a = sm.ka[i], qp = sm.qtp[i];
-            r4.x = fmaf(a, S[m].x, r4.x); r4.y = fmaf(a, S[m].y, r4.y);
-            r4.z = fmaf(a, S[m].z, r4.z); r4.w = fmaf(a, S[m].w, r4.w);
-            o4.x = fmaf(qp, S[m].x, o4.x); o4.y = fmaf(qp, S[m].y, o4.y);
-            o4.z = fmaf(qp, S[m].z, o4.z); o4.w = fmaf(qp, S[m].w, o4.w);
-        }
-        *reinterpret_cast<float4 *>(&sm.redA[2 * warp + hl][col4]) = r4;
-        if (o_tok >= 0) *reinterpret_cast<float4 *>(&sm.redB[2 * warp + hl][col4]) = o4;
-        __syncthreads();
-        if (tid < kBH) {
-            float s = 0.f;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) s += sm.redA[u][tid];
-            sm.r[tid] = s;
-            if (o_tok >= 0) {                                  // warps 0 and 1: this CTA's 64 columns of o
-                float oo = 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) oo += sm.redB[u][tid];
-                const float ss = warp_sum(oo * oo), cs = warp_sum(sm.gdyp[tid] * oo);
-                if (lane == 0)
-                    *reinterpret_cast<float2 *>(part + (size_t)o_tok * 8 + 2 * (2 * c + warp)) = make_float2(ss, cs);
-            }
-        }
-        __syncthreads();
-        if (!update) return;
-        const float4 rr = ld4(&sm.r[col4]), vv = ld4(&sm.vh[col4]);
-#pragma unroll
-        for (int m = 0; m < kBRows; ++m) {
-            const int i = row_of(m);
-            const float al = sm.al[i], kh = sm.kh[i], kk = sm.k[i];
-            S[m].x = al * S[m].x - kh * rr.x + kk * vv.x;
-            S[m].y = al * S[m].y - kh * rr.y + kk * vv.y;
-            S[m].z = al * S[m].z - kh * rr.z + kk * vv.z;
-            S[m].w = al * S[m].w - kh * rr.w + kk * vv.w;
+            const float al = bf.al[i], kh = bf.kh[i], kk = bf.k[i];
+            S[m].x = state_step(S[m].x, al, kh, rr.x, kk, vv.x);
+            S[m].y = state_step(S[m].y, al, kh, rr.y, kk, vv.y);
+            S[m].z = state_step(S[m].z, al, kh, rr.z, kk, vv.z);
+            S[m].w = state_step(S[m].w, al, kh, rr.w, kk, vv.w);
         }
     };
+    // warps 4-5: o of token to (column j) from the 16 partials in redB, written to
+    // the workspace with this warp's RMS partials (g*dy of that token: gdy)
+    auto finish_o = [&](int to, float gdy) {
+        float oo = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) oo += sm.redB[u][j];
+        orw[(size_t)to * 2 * kBH + j] = oo;
+        const float ss = warp_sum(oo * oo), cs = warp_sum(gdy * oo);
+        if (lane == 0) *reinterpret_cast<float2 *>(part + (size_t)to * 8 + 2 * (2 * c + warp - 4)) = make_float2(ss, cs);
+    };
 
-    // ---- phase F: checkpoints S_0, S_kBC, S_2kBC, ... and the RMS partials of every token
+    // ---- phase F: checkpoints S_0, S_kBC, S_2kBC, ..., and per token o, r and
+    // the RMS partials.  Two barriers a token: after the staging, and after the
+    // column partials of r_t = (k alpha) S_{t-1} and o_{t-1} = q~_{t-1} S_{t-1}.
+    // Every thread then sums the partials of its own four columns of r itself.
     {
         float4 S[kBRows];
         const float *s_in = p.S_in ? p.S_in + (size_t)head * kBD * kBD : nullptr;
 #pragma unroll
         for (int m = 0; m < kBRows; ++m) S[m] = s_in ? ld4(s_in + own_full(m)) : make_float4(0.f, 0.f, 0.f, 0.f);
         store_rows(ckpt, S);
-        Tok c0 = T_ > 0 ? fetch(0, false) : Tok{}, c1 = T_ > 1 ? fetch(1, false) : Tok{};
-        for (int t = 0; t < T_; ++t) {
+        Tok c0 = T_ > 0 ? fetch(0, kF) : Tok{}, c1 = T_ > 1 ? fetch(1, kF) : Tok{};
+        Tok c2 = T_ > 2 ? fetch(2, kF) : Tok{}, c3 = T_ > 3 ? fetch(3, kF) : Tok{};
+        float gdy_prev = 0.f;                                 // value threads: g*dy of the previous token
+        // token t from cx, which then takes token t + 4's inputs (four register
+        // sets, used in turn, so that no move waits for a load in flight)
+        auto f_token = [&](int t, Tok &cx) {
+            TokBuf &cb = sm.tb[t & 1];
+            const TokBuf &pb = sm.tb[(t & 1) ^ 1];
+            stage(cx, kF, cb);
+            const float gdy_cur = cv(cx.v3) * dy_of(cx);
+            if (t + 4 < T_) cx = fetch(t + 4, kF);
             __syncthreads();
-            stage(c0, true, false);
-            c0 = c1;
-            if (t + 2 < T_) c1 = fetch(t + 2, false);
+            {
+                float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f), o4 = r4;
+#pragma unroll
+                for (int m = 0; m < kBRows; ++m) {
+                    const int i = row_of(m);
+                    const float a = cb.ka[i];
+                    r4.x = fmaf(a, S[m].x, r4.x); r4.y = fmaf(a, S[m].y, r4.y);
+                    r4.z = fmaf(a, S[m].z, r4.z); r4.w = fmaf(a, S[m].w, r4.w);
+                }
+                *reinterpret_cast<float4 *>(&sm.redA[2 * warp + hl][col4]) = r4;
+                if (t > 0) {
+#pragma unroll
+                    for (int m = 0; m < kBRows; ++m) {
+                        const float qp = pb.qt[row_of(m)];
+                        o4.x = fmaf(qp, S[m].x, o4.x); o4.y = fmaf(qp, S[m].y, o4.y);
+                        o4.z = fmaf(qp, S[m].z, o4.z); o4.w = fmaf(qp, S[m].w, o4.w);
+                    }
+                    *reinterpret_cast<float4 *>(&sm.redB[2 * warp + hl][col4]) = o4;
+                }
+            }
             __syncthreads();
-            fwd_step(S, t - 1, true);                          // r of token t, o of token t - 1
+            float4 rr = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float4 a = ld4(&sm.redA[u][col4]);
+                rr.x += a.x; rr.y += a.y; rr.z += a.z; rr.w += a.w;
+            }
+            if (valt) {
+                float rj = 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) rj += sm.redA[u][j];
+                orw[(size_t)t * 2 * kBH + kBH + j] = rj;
+                if (t > 0) finish_o(t - 1, gdy_prev);
+                gdy_prev = gdy_cur;
+            }
+            update(S, cb, rr);
             if ((t + 1) % kBC == 0 && (t + 1) / kBC < NC) store_rows(ckpt + (size_t)((t + 1) / kBC) * mat, S);
+        };
+        for (int t = 0; t < T_; t += 4) {
+            f_token(t, c0);
+            if (t + 1 < T_) f_token(t + 1, c1);
+            if (t + 2 < T_) f_token(t + 2, c2);
+            if (t + 3 < T_) f_token(t + 3, c3);
         }
         if (T_ > 0) {                                          // o of the last token
+            const TokBuf &lb = sm.tb[(T_ - 1) & 1];
+            float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m = 0; m < kBRows; ++m) {
+                const float qp = lb.qt[row_of(m)];
+                o4.x = fmaf(qp, S[m].x, o4.x); o4.y = fmaf(qp, S[m].y, o4.y);
+                o4.z = fmaf(qp, S[m].z, o4.z); o4.w = fmaf(qp, S[m].w, o4.w);
+            }
+            __syncthreads();                                   // warps 4-5 are done with redB
+            *reinterpret_cast<float4 *>(&sm.redB[2 * warp + hl][col4]) = o4;
             __syncthreads();
-            if (tid < kBD) sm.qtp[tid] = sm.qt[tid];
-            else if (tid < kBD + kBH) sm.gdyp[tid - kBD] = sm.gdy[tid - kBD];
-            __syncthreads();
-            fwd_step(S, T_ - 1, false);
+            if (valt) finish_o(T_ - 1, gdy_prev);
         }
     }
-    // both CTAs' RMS partials are in the workspace before either reads them
+    // both CTAs' RMS partials are in the workspace before either reads them; the
+    // checkpoints are visible to the bulk copies that read state 0 of each chunk
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     __threadfence();
     tc::cluster_sync();
 
@@ -245,74 +361,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     float dgam = 0.f;                                          // this CTA's share of d gamma_stat, channel tid (tid < 128)
     for (int ch = NC - 1; ch >= 0; --ch) {
         const int t0 = ch * kBC, t1 = min(T_, t0 + kBC);
-        {   // the chunk's states S_{t0} .. S_{t1}
-            float4 S[kBRows];
+        // The chunk's states: state s is S before token t0 + s (state 0 is the
+        // checkpoint), s = 0 .. n.  The recompute (one barrier a token, with each
+        // token's r from phase F) writes each state to slot s & 1; states 1 .. n-2
+        // go on to the chunk buffer.  The walk keeps state n in registers, finds
+        // state n-1 still in its slot and loads states n-2 .. 0 back one token
+        // ahead (state 0 from the checkpoint).
+        const int n = t1 - t0;
+        float4 S[kBRows];
+        {
             load_rows(ckpt + (size_t)ch * mat, S);
-            store_rows(chunk, S);
-            Tok c0 = fetch(t0, false), c1 = t0 + 1 < t1 ? fetch(t0 + 1, false) : Tok{};
-            for (int t = t0; t < t1; ++t) {
+            store_rows(slot(0), S);
+            Tok c0 = fetch(t0, kRe), c1 = t0 + 1 < t1 ? fetch(t0 + 1, kRe) : Tok{};
+            Tok c2 = t0 + 2 < t1 ? fetch(t0 + 2, kRe) : Tok{}, c3 = t0 + 3 < t1 ? fetch(t0 + 3, kRe) : Tok{};
+            auto r_token = [&](int t, Tok &cx) {
+                const int st = t - t0 + 1;                     // the state this token makes
+                TokBuf &cb = sm.tb[t & 1];
+                stage(cx, kRe, cb);
+                if (t + 4 < t1) cx = fetch(t + 4, kRe);
+                if (tid == 0) tc::bulk_wait_read();            // slot st & 1 has been read out
                 __syncthreads();
-                stage(c0, false, false);
-                c0 = c1;
-                if (t + 2 < t1) c1 = fetch(t + 2, false);
-                __syncthreads();
-                fwd_step(S, -1, true);
-                store_rows(chunk + (size_t)(t - t0 + 1) * mat, S);
+                if (tid == 0 && st - 1 >= 1 && st - 1 <= n - 2) {
+                    tc::bulk_s2g(chunk + (size_t)(st - 1) * mat, s_slot0 + ((st - 1) & 1) * kSlotBytes, kSlotBytes);
+                    tc::bulk_commit();
+                }
+                update(S, cb, ld4(&cb.r[col4]));
+                store_rows(slot(st & 1), S);
+                tc::fence_proxy_async();
+            };
+            for (int t = t0; t < t1; t += 4) {
+                r_token(t, c0);
+                if (t + 1 < t1) r_token(t + 1, c1);
+                if (t + 2 < t1) r_token(t + 2, c2);
+                if (t + 3 < t1) r_token(t + 3, c3);
             }
         }
-        Tok n0 = fetch(t1 - 1, true), n1 = t1 - 2 >= t0 ? fetch(t1 - 2, true) : Tok{};
+        Tok n0 = fetch(t1 - 1, kWalk), n1 = t1 - 2 >= t0 ? fetch(t1 - 2, kWalk) : Tok{};
         // this thread's rows of S_t and S_{t-1}, held in registers for the whole
-        // token; walking backward, S_{t-1} of one token is S_t of the next, so each
-        // token loads one state (issued before its barriers)
+        // token; walking backward, S_{t-1} of one token is S_t of the next
         float4 stv[kBRows], spv[kBRows];
-        load_rows(chunk + (size_t)(t1 - t0) * mat, stv);
-        for (int t = t1 - 1; t >= t0; --t) {
-            load_rows(chunk + (size_t)(t - t0) * mat, spv);
-            __syncthreads();
-            const Tok cur = n0;                                // token t (also read by steps 2, 4 and 6)
-            stage(cur, false, true);
-            n0 = n1;
-            if (t - 2 >= t0) n1 = fetch(t - 2, true);
-            __syncthreads();
+#pragma unroll
+        for (int m = 0; m < kBRows; ++m) stv[m] = S[m];
+        if (tid == 0) tc::bulk_wait_all();                     // the chunk buffer holds states 1 .. n-2
+        __syncthreads();                                       // the recompute's last token is read before it is staged again
+        auto w_token = [&](int t, Tok &cx) {
+            const int st = t - t0;                             // S_{t-1} is state st
+            if (tid == kLoader && st >= 1) {                   // state st - 1, for the next token
+                const int x = (st - 1) & 1;
+                const float *src = st - 1 == 0 ? ckpt + (size_t)ch * mat : chunk + (size_t)(st - 1) * mat;
+                tc::fence_proxy_async();
+                tc::mbar_arrive_expect_tx(s_mb + 8 * x, kSlotBytes);
+                tc::bulk_g2s(s_slot0 + x * kSlotBytes, src, kSlotBytes, s_mb + 8 * x);
+            }
+            TokBuf &cb = sm.tb[t & 1];
+            const Tok cur = cx;                                // token t (also read by steps 4 and 6)
             const size_t gt = ((size_t)bb * T_ + t) * H + h;
-            // (1) o = q~ S_t and r = (k alpha) S_{t-1}: column partials
-            {
-                float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f), r4 = o4;
-#pragma unroll
-                for (int m = 0; m < kBRows; ++m) {
-                    const int i = row_of(m);
-                    const float4 st = stv[m], sp = spv[m];
-                    const float a = sm.qt[i], c2 = sm.ka[i];
-                    o4.x = fmaf(a, st.x, o4.x); o4.y = fmaf(a, st.y, o4.y);
-                    o4.z = fmaf(a, st.z, o4.z); o4.w = fmaf(a, st.w, o4.w);
-                    r4.x = fmaf(c2, sp.x, r4.x); r4.y = fmaf(c2, sp.y, r4.y);
-                    r4.z = fmaf(c2, sp.z, r4.z); r4.w = fmaf(c2, sp.w, r4.w);
-                }
-                *reinterpret_cast<float4 *>(&sm.redA[2 * warp + hl][col4]) = o4;
-                *reinterpret_cast<float4 *>(&sm.redB[2 * warp + hl][col4]) = r4;
+            stage(cur, kWalk, cb);
+            // (2) the value side of column j: the RMS norm over both CTAs' columns
+            // (the four partial pairs, summed in a fixed order), do and dg
+            if (valt) {
+                const float ss = ((cur.pa.x + cur.pa.z) + cur.pb.x) + cur.pb.z;
+                const float cs = ((cur.pa.y + cur.pa.w) + cur.pb.y) + cur.pb.w;
+                const float rho = rsqrtf(ss / kBD + p.eps), oo = fl(cur.v5), dyv = dy_of(cur);
+                cb.dO[j] = rho * (cv(cur.v3) * dyv) - rho * rho * rho / kBD * oo * cs;
+                p.grad_g[gt * kBD + gc0 + j] = dyv * oo * rho;
             }
-            __syncthreads();
-            // (2) the value side of column j: o and r, the RMS norm over both CTAs'
-            // columns (the four partial pairs, summed in a fixed order), do and dg
-            if (tid >= kBD && tid < kBD + kBH) {
-                const int j = tid - kBD;
-                float oo = 0.f, sr = 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    oo += sm.redA[u][j];
-                    sr += sm.redB[u][j];
-                }
-                sm.r[j] = sr;
-                const float *pp = reinterpret_cast<const float *>(sm.part);
-                const float ss = ((pp[0] + pp[2]) + pp[4]) + pp[6], cs = ((pp[1] + pp[3]) + pp[5]) + pp[7];
-                const float rho = rsqrtf(ss / kBD + p.eps);
-                sm.dO[j] = rho * sm.gdy[j] - rho * rho * rho / kBD * oo * cs;
-                p.grad_g[gt * kBD + gc0 + j] = cur.x2 * oo * rho;
-            }
+            if (t - 2 >= t0) cx = fetch(t - 2, kWalk);
             __syncthreads();
             // (3) dS += q~^T do; dq~ = S_t do^T (rows); k dS and (b*k) dS (columns)
             {
-                const float4 d4 = ld4(&sm.dO[col4]);
+                const float4 d4 = ld4(&cb.dO[col4]);
                 float rowv[kBRows];
                 float4 cA = make_float4(0.f, 0.f, 0.f, 0.f), cB = cA;
 #pragma unroll
@@ -321,11 +439,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                     const float4 st = stv[m];
                     rowv[m] = dot4(st, d4);
                     float4 ds = sdS[i * 16 + lc];
-                    const float a = sm.qt[i];
+                    const float a = cb.qt[i];
                     ds.x = fmaf(a, d4.x, ds.x); ds.y = fmaf(a, d4.y, ds.y);
                     ds.z = fmaf(a, d4.z, ds.z); ds.w = fmaf(a, d4.w, ds.w);
                     sdS[i * 16 + lc] = ds;
-                    const float kk = sm.k[i], kh = sm.kh[i];
+                    const float kk = cb.k[i], kh = cb.kh[i];
                     cA.x = fmaf(kk, ds.x, cA.x); cA.y = fmaf(kk, ds.y, cA.y);
                     cA.z = fmaf(kk, ds.z, cA.z); cA.w = fmaf(kk, ds.w, cA.w);
                     cB.x = fmaf(kh, ds.x, cB.x); cB.y = fmaf(kh, ds.y, cB.y);
@@ -338,8 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
             }
             __syncthreads();
             // (4) dv^ and dr on this CTA's columns; dv, dw
-            if (tid >= kBD && tid < kBD + kBH) {
-                const int j = tid - kBD;
+            if (valt) {
                 float sa = 0.f, sb = 0.f;
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -348,13 +465,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                 }
                 sm.dr[j] = -sb;
                 const size_t gj = gt * kBD + gc0 + j;
-                p.grad_v[gj] = cur.x0 * sa;
-                p.grad_w[gj] = cur.x1 * sa;
+                p.grad_v[gj] = cv(cur.v0) * sa;
+                p.grad_w[gj] = cv(cur.v1) * sa;
             }
             __syncthreads();
             // (5) row sums dS v^T, -dS r^T, S_{t-1} dr^T, (dS + k^T dr) * S_{t-1}; dS <- Diag(alpha) dS_hat
+            if (st <= n - 2) wait_slot(st & 1);
+            load_rows(slot(st & 1), spv);
             {
-                const float4 vv = ld4(&sm.vh[col4]), rr = ld4(&sm.r[col4]), dd = ld4(&sm.dr[col4]);
+                const float4 vv = ld4(&cb.vh[col4]), rr = ld4(&cb.r[col4]), dd = ld4(&sm.dr[col4]);
                 float ra[kBRows], rb[kBRows], rc[kBRows], rd[kBRows];
 #pragma unroll
                 for (int m = 0; m < kBRows; ++m) {
@@ -364,7 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                     ra[m] = dot4(ds, vv);
                     rb[m] = -dot4(ds, rr);
                     rc[m] = dot4(sp, dd);
-                    const float kk = sm.k[i], al = sm.al[i];
+                    const float kk = cb.k[i], al = cb.al[i];
                     ds.x = fmaf(kk, dd.x, ds.x); ds.y = fmaf(kk, dd.y, ds.y);
                     ds.z = fmaf(kk, dd.z, ds.z); ds.w = fmaf(kk, dd.w, ds.w);
                     rd[m] = dot4(ds, sp);
@@ -383,21 +502,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
             }
             __syncthreads();
             // (6) this CTA's share of token t's key-side gradients (the other CTA adds its share)
-            if (tid < kBD) {
+            if (keyt) {
                 const size_t gi = gt * kBD + tid;
-                const float kk = sm.k[tid], al = sm.al[tid];
-                const float bv = cur.x2, qv = cur.x3, zv = cur.x4;
+                const float kk = cb.k[tid], al = cb.al[tid];
+                const float bv = cv(cur.k2), qv = cv(cur.k3), zv = cv(cur.k4);
                 const float ts = two_sigmoid(zv);
                 const float dqt = sm.rows[0][tid], dkh = sm.rows[2][tid];
-                atomicAdd(p.grad_k + gi, sm.rows[1][tid] + al * sm.rows[3][tid] + bv * dkh);
-                atomicAdd(p.grad_b + gi, kk * dkh);
-                atomicAdd(p.grad_la + gi, al * sm.rows[4][tid]);
-                atomicAdd(p.grad_q + gi, dqt * gs_own * ts);
-                atomicAdd(p.grad_z + gi, dqt * qv * gs_own * ts * (1.f - 0.5f * ts));
+                red_add(p.grad_k + gi, sm.rows[1][tid] + al * sm.rows[3][tid] + bv * dkh);
+                red_add(p.grad_b + gi, kk * dkh);
+                red_add(p.grad_la + gi, al * sm.rows[4][tid]);
+                red_add(p.grad_q + gi, dqt * gs_own * ts);
+                red_add(p.grad_z + gi, dqt * qv * gs_own * ts * (1.f - 0.5f * ts));
                 dgam = fmaf(dqt * qv, ts, dgam);
             }
 #pragma unroll
             for (int m = 0; m < kBRows; ++m) stv[m] = spv[m];
+        };
+        for (int t = t1 - 1; t >= t0; t -= 2) {
+            w_token(t, n0);
+            if (t - 1 >= t0) w_token(t - 1, n1);
         }
     }
     __syncthreads();
@@ -406,7 +529,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
         for (int m = 0; m < kBRows; ++m)
             *reinterpret_cast<float4 *>(p.grad_S_in + (size_t)head * kBD * kBD + own_full(m)) = sdS[row_of(m) * 16 + lc];
     }
-    if (tid < kBD) p.ws_dgam[hc * kBD + tid] = dgam;
+    if (keyt) p.ws_dgam[hc * kBD + tid] = dgam;
 }
 
 // d gamma_stat[h] = sum over the batch rows and both value halves of the per-CTA partials
@@ -424,7 +547,8 @@ size_t bwd_workspace_bytes(int B, int H, int T) {
     const size_t mat = (size_t)kBD * kBH * sizeof(float);          // one half-matrix
     const size_t NC = (size_t)(T + kBC - 1) / kBC;
     const size_t BH = (size_t)B * H;
-    return BH * 2 * ((NC + 1) * mat + (kBC + 1) * mat + kBD * sizeof(float)) + BH * (size_t)T * 8 * sizeof(float);
+    return BH * 2 * ((NC + 1) * mat + (kBC + 1) * mat + kBD * sizeof(float)) + BH * (size_t)T * 8 * sizeof(float) +
+           BH * 2 * (size_t)T * 2 * kBH * sizeof(float);
 }
 
 cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t stream) {
@@ -436,6 +560,7 @@ cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t str
     p.ws_chunk = p.ws_ckpt + BH * 2 * (NC + 1) * mat;
     p.ws_dgam = p.ws_chunk + BH * 2 * (kBC + 1) * mat;
     p.ws_part = p.ws_dgam + BH * 2 * kBD;
+    p.ws_or = p.ws_part + BH * (size_t)p.T * 8;
     // the key-side gradients are accumulated by the two CTAs of each head
     const size_t ntok = BH * (size_t)p.T * kBD * sizeof(float);
     cudaError_t e = cudaSuccess;
@@ -446,7 +571,8 @@ cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t str
             if (e != cudaSuccess) return e;
         }
     }
-    const size_t dsm = (size_t)kBD * kBH * sizeof(float);           // running dS of one CTA's columns
+    // running dS of one CTA's columns, two state tiles, their mbarriers
+    const size_t dsm = (size_t)kBD * kBH * sizeof(float) + 2 * (size_t)kSlotBytes + 16;
     if (dtype == GDELTA_BF16) {
         e = cudaFuncSetAttribute(gdn2_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm);
         if (e != cudaSuccess) return e;

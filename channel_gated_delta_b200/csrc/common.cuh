@@ -83,7 +83,9 @@ struct BwdParams {
     const float *dy, *dS_out;
     float eps;
     float *grad_q, *grad_k, *grad_v, *grad_b, *grad_w, *grad_z, *grad_g, *grad_la, *grad_gs, *grad_S_in;
-    float *ws_ckpt, *ws_chunk, *ws_dgam, *ws_part;
+    float *ws_ckpt, *ws_chunk, *ws_dgam, *ws_part, *ws_or;
+    int *status;             // device status word (a bounded wait that ran out)
+    uint32_t wait_limit;     // polls before such a wait gives up
 };
 
 // Five-gate low-rank projection (gdelta.h, gdelta_gate_proj).

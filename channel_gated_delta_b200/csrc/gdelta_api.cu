@@ -172,6 +172,8 @@ gdelta_status gdelta_bwd(const gdelta_bwd_args *a, void *stream) {
     p.grad_q = a->grad_q; p.grad_k = a->grad_k; p.grad_v = a->grad_v; p.grad_b = a->grad_b;
     p.grad_w = a->grad_w; p.grad_z = a->grad_z; p.grad_g = a->grad_g; p.grad_la = a->grad_log_alpha;
     p.grad_gs = a->grad_gamma_stat; p.grad_S_in = a->grad_S_in;
+    p.status = status_ptr();
+    p.wait_limit = g_wait_polls.load(std::memory_order_relaxed);
     return launch_bwd(p, a->workspace, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
                                                                                     : GDELTA_ERR_CUDA;
 }

@@ -238,8 +238,9 @@ GDELTA_API gdelta_status gdelta_state_affine(float *S_out, const float *A, const
  *   grad_S_in       : [B, H, d_k, d_v] fp32 out or NULL
  *   workspace       : gdelta_bwd_workspace_bytes(args) bytes of device memory
  *                     (checkpoints and one chunk of states per head and value
- *                     half, and two RMS partial sums per token, head and
- *                     warp-pair);
+ *                     half, two RMS partial sums per token, head and
+ *                     warp-pair, and per token, head and value half the
+ *                     token's o and r on that half's columns);
  *                     GDELTA_ERR_WORKSPACE if smaller
  * Unsupported shapes return GDELTA_ERR_UNSUPPORTED.  Asynchronous on `stream`.
  */

@@ -152,7 +152,8 @@ def test_backward_validation(lib):
     need = wsb(ctypes.byref(_bwd_args()))
     # per value half of the head: checkpoints (2 for 64 tokens, plus one spare) and
     # 33 chunk states of 32 KiB, and 128 floats; per token: 8 floats of RMS partials
-    assert need == 2 * ((3 + 33) * 128 * 64 * 4 + 128 * 4) + 64 * 8 * 4
+    # and, per value half, the token's o and r on that half's 64 columns
+    assert need == 2 * ((3 + 33) * 128 * 64 * 4 + 128 * 4) + 64 * 8 * 4 + 2 * 64 * 128 * 4
     assert f(ctypes.byref(_bwd_args(workspace=0x900000, workspace_bytes=need - 1)), None) == 6
     assert wsb(ctypes.byref(_bwd_args(dk=64))) == 0
     # no tokens: token tensors may be null
