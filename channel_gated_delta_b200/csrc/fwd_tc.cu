@@ -1295,29 +1295,37 @@ __global__ void __launch_bounds__(kThreads, 3)
         // log-decays for the cross-warp prefix; the build below reads them again token
         // by token (from L2, one token ahead) and keeps only a running sum.
         const int tb = 8 * warp, c4 = 4 * lane;
-        auto gt_of = [&](int u) -> size_t { return ((size_t)bb * T + t0 + tb + u) * H + h; };
-        auto load_la = [&](int u) -> float4 {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t0 + tb + u < wend) {
-                if (kTok) {
-                    const float sc = __ldg(p.la + gt_of(u));
-                    x = make_float4(sc, sc, sc, sc);
-                } else {
-                    x = __ldg(reinterpret_cast<const float4 *>(p.la + gt_of(u) * kDK + c4));
-                }
-            }
+        // Look-ahead loads are unconditional, from the token index clamped into the
+        // window, and keep their raw bits; the zeros past the end of the sequence
+        // and any broadcast are applied where the value is used.  (A load whose
+        // result is selected against a zero, or shifted, right away makes the warp
+        // wait for it there, which defeats loading it ahead.)
+        auto live = [&](int u) { return t0 + tb + u < wend; };
+        auto gtc_of = [&](int u) -> size_t { return ((size_t)bb * T + min(t0 + tb + u, wend - 1)) * H + h; };
+        auto load_la = [&](int u) -> float4 {       // kTok: the token's scalar in .x
+            float4 x;
+            if (kTok) x.x = __ldg(p.la + gtc_of(u));
+            else x = __ldg(reinterpret_cast<const float4 *>(p.la + gtc_of(u) * kDK + c4));
             return x;
         };
-        // token u's beta, when b comes per token (zeros past the end of the sequence)
-        auto load_beta = [&](int u) -> uint2 {
-            return kBeta && t0 + tb + u < wend ? bf16x4_bcast(p.beta, gt_of(u)) : make_uint2(0, 0);
+        auto la_val = [&](float4 x, int u) -> float4 {
+            if (kTok) x = make_float4(x.x, x.x, x.x, x.x);
+            return live(u) ? x : make_float4(0.f, 0.f, 0.f, 0.f);
+        };
+        // token u's beta, when b comes per token: the raw bf16, then as a quad
+        auto load_beta = [&](int u) -> uint32_t {
+            return kBeta ? (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p.beta) + gtc_of(u)) : 0u;
+        };
+        auto beta_val = [&](uint32_t x, int u) -> uint2 {
+            const uint32_t q2 = live(u) ? (x | (x << 16)) : 0u;
+            return make_uint2(q2, q2);
         };
         float off[4] = {0.f, 0.f, 0.f, 0.f};
         {
             float tot[4] = {0.f, 0.f, 0.f, 0.f}, first[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float4 x = load_la(u);
+                const float4 x = la_val(load_la(u), u);
                 if (u == 0) {
                     first[0] = x.x * kLog2e; first[1] = x.y * kLog2e; first[2] = x.z * kLog2e; first[3] = x.w * kLog2e;
                 }
@@ -1380,27 +1388,26 @@ __global__ void __launch_bounds__(kThreads, 3)
             }
             float lam_run[4] = {off[0], off[1], off[2], off[3]};     // Lambda before token u
             float4 la_nx = load_la(0);
-            uint2 beta_nx = load_beta(0);
+            uint32_t beta_nx = load_beta(0);
             float dg[16];                             // [u]: q~.k, [8+u]: q~.(b*k) of token tb+u, this lane's channels
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = tb + u;
-                const bool live = t < n;
-                const float4 la_c = la_nx;
+                const bool live_t = t < n;
+                const float4 la_c = la_val(la_nx, u);
+                const uint2 beta_c = beta_val(beta_nx, u);
                 const uint32_t off_t = tc::tile_off(128, t, c4), off_b = tc::tile_off(128, 64 + t, c4);
                 // this thread's four channels of the raw k, q, z, b (their tile places)
                 const uint2 kq_c[4] = {*(const uint2 *)(sm + L::AP + off_t), *(const uint2 *)(sm + L::AP + off_b),
                                        kNoZ ? make_uint2(0, 0) : *(const uint2 *)(sm + L::BP + off_t),
-                                       kBeta ? beta_nx : *(const uint2 *)(sm + L::BP + off_b)};
+                                       kBeta ? beta_c : *(const uint2 *)(sm + L::BP + off_b)};
                 if (u + 1 < 8) {                      // the next token's log-decay is in flight meanwhile
                     la_nx = load_la(u + 1);
                     beta_nx = load_beta(u + 1);
-                } else {
-                    const bool in = t0 + tb < wend;   // the value side of token 0, for after the build
-                    const size_t gt = gt_of(0), gv = gt * kDV + c4;
-                    vw_nx[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                    vw_nx[1] = !in ? make_uint2(0, 0)
-                               : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                } else {                              // the value side of token 0, for after the build
+                    const size_t gt = gtc_of(0), gv = gt * kDV + c4;
+                    vw_nx[0] = __ldg(reinterpret_cast<const uint2 *>(p.v + gv));
+                    vw_nx[1] = kBeta ? make_uint2(load_beta(0), 0u) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
                 }
                 lam_run[0] += la_c.x * kLog2e; lam_run[1] += la_c.y * kLog2e;
                 lam_run[2] += la_c.z * kLog2e; lam_run[3] += la_c.w * kLog2e;
@@ -1427,11 +1434,11 @@ __global__ void __launch_bounds__(kThreads, 3)
                 float dq = 0.f, db = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float lam = live ? lam_run[c] : lnv[c];
+                    const float lam = live_t ? lam_run[c] : lnv[c];
                     const float d = lam - cpiv[c];
                     const float ep = ex2(d), em = ex2(-d);
-                    const float kv = live ? kk[c] : 0.f;
-                    const float qt = live ? qq[c] * gq[c] * two_sigmoid_fast(zz[c]) : 0.f;
+                    const float kv = live_t ? kk[c] : 0.f;
+                    const float qt = live_t ? qq[c] * gq[c] * two_sigmoid_fast(zz[c]) : 0.f;
                     const float kh = bv[c] * kv;
                     dq += qt * kv;
                     db += qt * kh;
@@ -1481,13 +1488,13 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int t = tb + u;
-            const uint2 vw_c[2] = {vw_nx[0], vw_nx[1]};
+            const bool in = live(u);
+            const uint2 vw_c[2] = {in ? vw_nx[0] : make_uint2(0, 0),
+                                   !in ? make_uint2(0, 0) : kBeta ? beta_val(vw_nx[1].x, u) : vw_nx[1]};
             if (u + 1 < 8) {
-                const bool in = t0 + t + 1 < wend;
-                const size_t gt = gt_of(u + 1), gv = gt * kDV + c4;
-                vw_nx[0] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + gv)) : make_uint2(0, 0);
-                vw_nx[1] = !in ? make_uint2(0, 0)
-                           : kBeta ? bf16x4_bcast(p.beta, gt) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+                const size_t gt = gtc_of(u + 1), gv = gt * kDV + c4;
+                vw_nx[0] = __ldg(reinterpret_cast<const uint2 *>(p.v + gv));
+                vw_nx[1] = kBeta ? make_uint2(load_beta(u + 1), 0u) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
             }
             const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
             const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
