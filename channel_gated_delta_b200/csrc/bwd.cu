@@ -40,7 +40,7 @@
 // and the chain rule through q~ = q * gamma * 2 sigmoid(z), v^ = w * v,
 // alpha = exp(log_alpha).  The checkpoints, chunk states, per-token o and r and
 // RMS partials live in the caller's workspace; the running dS (this CTA's half)
-// lives in shared memory.
+// lives in registers, each thread holding its own elements.
 //
 // Thread layout (256 threads): warp w, lane l = 16 h + c holds rows
 // w + 8 h + 16 m (m = 0..7) and the CTA's columns 4c..4c+3, so a row's sum over
@@ -129,7 +129,7 @@ __device__ __forceinline__ float state_step(float s, float al, float kh, float r
 template <typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_kernel(BwdParams p) {
     __shared__ BwdSmem sm;
-    extern __shared__ float4 sdS[];                          // running dS of this CTA's columns, [row][16]
+    extern __shared__ float4 dsm_base[];                     // two state tiles, then their mbarriers
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hl = lane >> 4, lc = lane & 15, col4 = 4 * lc;
     const int c = (int)tc::cluster_ctarank(), gc0 = kBH * c;  // this CTA's first value column
@@ -150,10 +150,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     auto own = [&](int m) { return (size_t)row_of(m) * kBH + col4; };           // in a half-matrix buffer
     auto own_full = [&](int m) { return (size_t)row_of(m) * kBD + gc0 + col4; };  // in a [128][128] matrix
     // Two state tiles in shared memory (each a [128][64] half-matrix, the chunk
-    // buffer's layout) and their mbarriers, after the running dS.  The chunk's
+    // buffer's layout) and their mbarriers.  The chunk's
     // states move between them and the chunk buffer by bulk copies (one thread,
     // 32 KiB each), which keeps that traffic off the threads' load/store path.
-    float *const slot0 = reinterpret_cast<float *>(sdS + kBD * 16);
+    float *const slot0 = reinterpret_cast<float *>(dsm_base);
     auto slot = [&](int x) { return slot0 + (size_t)x * mat; };
     const uint32_t s_slot0 = tc::smem_u32(slot0), s_mb = s_slot0 + 2 * kSlotBytes;
     uint32_t ph = 0;                                          // bit x: parity of the next wait on slot x
@@ -351,12 +351,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     __threadfence();
     tc::cluster_sync();
 
-    // ---- phase B
+    // ---- phase B.  The running dS of this thread's elements (its rows, its four
+    // columns) stays in registers: no other thread reads them.
+    float4 dS[kBRows];
     {
         const float *ds_out = p.dS_out ? p.dS_out + (size_t)head * kBD * kBD : nullptr;
 #pragma unroll
-        for (int m = 0; m < kBRows; ++m)
-            sdS[row_of(m) * 16 + lc] = ds_out ? ld4(ds_out + own_full(m)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < kBRows; ++m) dS[m] = ds_out ? ld4(ds_out + own_full(m)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     float dgam = 0.f;                                          // this CTA's share of d gamma_stat, channel tid (tid < 128)
     for (int ch = NC - 1; ch >= 0; --ch) {
@@ -438,11 +439,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                     const int i = row_of(m);
                     const float4 st = stv[m];
                     rowv[m] = dot4(st, d4);
-                    float4 ds = sdS[i * 16 + lc];
+                    float4 ds = dS[m];
                     const float a = cb.qt[i];
                     ds.x = fmaf(a, d4.x, ds.x); ds.y = fmaf(a, d4.y, ds.y);
                     ds.z = fmaf(a, d4.z, ds.z); ds.w = fmaf(a, d4.w, ds.w);
-                    sdS[i * 16 + lc] = ds;
+                    dS[m] = ds;
                     const float kk = cb.k[i], kh = cb.kh[i];
                     cA.x = fmaf(kk, ds.x, cA.x); cA.y = fmaf(kk, ds.y, cA.y);
                     cA.z = fmaf(kk, ds.z, cA.z); cA.w = fmaf(kk, ds.w, cA.w);
@@ -479,7 +480,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                 for (int m = 0; m < kBRows; ++m) {
                     const int i = row_of(m);
                     const float4 sp = spv[m];
-                    float4 ds = sdS[i * 16 + lc];
+                    float4 ds = dS[m];
                     ra[m] = dot4(ds, vv);
                     rb[m] = -dot4(ds, rr);
                     rc[m] = dot4(sp, dd);
@@ -488,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                     ds.z = fmaf(kk, dd.z, ds.z); ds.w = fmaf(kk, dd.w, ds.w);
                     rd[m] = dot4(ds, sp);
                     ds.x *= al; ds.y *= al; ds.z *= al; ds.w *= al;
-                    sdS[i * 16 + lc] = ds;
+                    dS[m] = ds;
                 }
                 const int ri = row_of((lane >> 1) & 7);
                 const float sa = rows_reduce_scatter8(ra, lane), sb = rows_reduce_scatter8(rb, lane);
@@ -527,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     if (p.grad_S_in) {
 #pragma unroll
         for (int m = 0; m < kBRows; ++m)
-            *reinterpret_cast<float4 *>(p.grad_S_in + (size_t)head * kBD * kBD + own_full(m)) = sdS[row_of(m) * 16 + lc];
+            *reinterpret_cast<float4 *>(p.grad_S_in + (size_t)head * kBD * kBD + own_full(m)) = dS[m];
     }
     if (keyt) p.ws_dgam[hc * kBD + tid] = dgam;
 }
@@ -571,8 +572,8 @@ cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t str
             if (e != cudaSuccess) return e;
         }
     }
-    // running dS of one CTA's columns, two state tiles, their mbarriers
-    const size_t dsm = (size_t)kBD * kBH * sizeof(float) + 2 * (size_t)kSlotBytes + 16;
+    // two state tiles and their mbarriers
+    const size_t dsm = 2 * (size_t)kSlotBytes + 16;
     if (dtype == GDELTA_BF16) {
         e = cudaFuncSetAttribute(gdn2_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm);
         if (e != cudaSuccess) return e;
