@@ -150,7 +150,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     auto own = [&](int m) { return (size_t)row_of(m) * kBH + col4; };           // in a half-matrix buffer
     auto own_full = [&](int m) { return (size_t)row_of(m) * kBD + gc0 + col4; };  // in a [128][128] matrix
     // Two state tiles in shared memory (each a [128][64] half-matrix, the chunk
-    // buffer's layout) and their mbarriers.  The chunk's
+    // buffer's layout) and their mbarriers (a third one is never completed: the
+    // failure-path test waits on it).  The chunk's
     // states move between them and the chunk buffer by bulk copies (one thread,
     // 32 KiB each), which keeps that traffic off the threads' load/store path.
     float *const slot0 = reinterpret_cast<float *>(dsm_base);
@@ -160,8 +161,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     if (tid == 0) {
         tc::mbar_init(s_mb, 1);
         tc::mbar_init(s_mb + 8, 1);
+        tc::mbar_init(s_mb + 16, 1);                          // never completed (failure-path tests)
     }
     __syncthreads();
+    // failure-path test: a wait that nothing completes runs out and is reported;
+    // both CTAs of the cluster leave here, before any cluster barrier
+    if (p.stall) {
+        if (tid == 0 && !tc::mbar_wait(s_mb + 16, 0, p.wait_limit) && p.status) atomicCAS(p.status, 0, (int)kDevTimeout);
+        return;
+    }
     // bounded wait for slot x's bulk load; a wait that runs out is reported and then
     // drained, so that no copy is still landing when the slot is used again
     auto wait_slot = [&](int x) {
@@ -572,8 +580,8 @@ cudaError_t launch_bwd(BwdParams p, void *workspace, int dtype, cudaStream_t str
             if (e != cudaSuccess) return e;
         }
     }
-    // two state tiles and their mbarriers
-    const size_t dsm = 2 * (size_t)kSlotBytes + 16;
+    // two state tiles and three mbarriers (the slots' and the failure-test one)
+    const size_t dsm = 2 * (size_t)kSlotBytes + 24;
     if (dtype == GDELTA_BF16) {
         e = cudaFuncSetAttribute(gdn2_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm);
         if (e != cudaSuccess) return e;

@@ -86,6 +86,7 @@ struct BwdParams {
     float *ws_ckpt, *ws_chunk, *ws_dgam, *ws_part, *ws_or;
     int *status;             // device status word (a bounded wait that ran out)
     uint32_t wait_limit;     // polls before such a wait gives up
+    int stall;               // 1: wait first on a barrier nothing completes, so that the wait runs out
 };
 
 // Five-gate low-rank projection (gdelta.h, gdelta_gate_proj).

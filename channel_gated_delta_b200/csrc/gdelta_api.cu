@@ -174,6 +174,7 @@ gdelta_status gdelta_bwd(const gdelta_bwd_args *a, void *stream) {
     p.grad_gs = a->grad_gamma_stat; p.grad_S_in = a->grad_S_in;
     p.status = status_ptr();
     p.wait_limit = g_wait_polls.load(std::memory_order_relaxed);
+    p.stall = g_stall_test.load(std::memory_order_relaxed);
     return launch_bwd(p, a->workspace, a->dtype, (cudaStream_t)stream) == cudaSuccess ? GDELTA_OK
                                                                                     : GDELTA_ERR_CUDA;
 }

@@ -362,8 +362,10 @@ GDELTA_API gdelta_status gdelta_gate_proj(const gdelta_gate_proj_args *args, voi
  * frees its tensor memory and returns.  polls = 0 restores the default of
  * 2^20 polls.  The setting is process-wide, read when a call is queued (calls
  * already queued keep their limit), and applies to gdelta_fwd_chunked and
- * gdelta_fwd_chunked_noalloc on the tensor-core path and to gdelta_gate_proj;
- * the other kernels do not wait.  A limit far below the time the hardware needs turns ordinary waits
+ * gdelta_fwd_chunked_noalloc on the tensor-core path, to gdelta_gate_proj and
+ * to gdelta_bwd (its waits for bulk copies of chunk states; a wait that runs
+ * out is reported and then drained with a fixed limit); the other kernels do
+ * not wait.  A limit far below the time the hardware needs turns ordinary waits
  * into timeouts: the call then reports GDELTA_ERR_TIMEOUT and its outputs are
  * unreliable, but the device stays usable.  Always returns GDELTA_OK.
  */

@@ -8,7 +8,8 @@ faulting the GPU.
   usable (the next call matches the oracle).
 * An fp16 operand out of range: keys scaled far beyond unit norm push the
   pivot-scaled operands past 6e4; the kernels must report GDELTA_ERR_RANGE.
-* The same bounded-wait failure in the five-gate projection kernel.
+* The same bounded-wait failure in the five-gate projection kernel and in the
+  backward pass.
 """
 import ctypes
 
@@ -115,3 +116,32 @@ def test_gate_projection_wait_that_runs_out(restore_failure_controls):
     from oracle import gate_proj as ogp
     ref = ogp.project(inp["x"].cpu(), inp["w_down"].cpu(), inp["w_up"].cpu(), inp["bias"].cpu())
     assert err(out["log_alpha"].cpu(), ref["log_alpha"]) <= TOL_BF16
+
+
+def test_backward_wait_that_runs_out_reports_timeout(restore_failure_controls):
+    """gdelta_bwd reports a bounded wait that runs out through the same status
+    word (both CTAs of each cluster leave before any cluster barrier), and the
+    next call matches the float64 autograd oracle."""
+    import channel_gated_delta_b200 as gd
+    from oracle import backward as ob
+    inp = synth.generate(synth.GdnShape(B=1, T=40, H=1, dk=128, dv=128, dtype="bf16", hot_channels=6, seed=21))
+    d = to_dev(inp)
+    dy = torch.randn(1, 40, 1, 128, generator=torch.Generator().manual_seed(21))
+
+    def call():
+        return gd.gdelta_bwd(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], dy.cuda(),
+                             gamma_stat=d["gamma_stat"])
+
+    assert gdelta_get_last_device_error() == 0
+    gdelta_set_wait_limit(64)
+    gdelta_set_wait_timeout_test(True)
+    call()
+    assert gdelta_get_last_device_error() == TIMEOUT
+    gdelta_set_wait_timeout_test(False)
+    gdelta_set_wait_limit(0)
+    g = call()
+    torch.cuda.synchronize()
+    assert gdelta_get_last_device_error() == 0
+    ref = ob.backward(inp, dy.numpy(), heads=oracle.all_heads(1, 1))
+    for key in ("q", "k", "v", "b", "w", "z", "g", "log_alpha"):
+        assert err(sel_heads(g[key].cpu(), oracle.all_heads(1, 1)), ref["d" + key]) <= 1e-4, key
