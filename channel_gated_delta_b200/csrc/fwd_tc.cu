@@ -1483,19 +1483,24 @@ __global__ void __launch_bounds__(kThreads, 3)
             tc::bulk_s2g(rec + kWinAP + 128 * 128 + 64 * 128, s_ap + 128 * 128 + 64 * 128, 64 * 128);  // columns 64-127
             tc::bulk_commit();
         }
-        // V^ = w*v -> window record (the identity padding past n is zero), token by
-        // token with the next token's v and w in flight, while the P product runs
+        // V^ = w*v -> window record (the identity padding past n is zero), while the P
+        // product runs: token 0's v and w were loaded during the build, the other
+        // seven tokens' are all issued here before the first is used
+        uint2 vr[8][2];
+        vr[0][0] = vw_nx[0];
+        vr[0][1] = vw_nx[1];
+#pragma unroll
+        for (int u = 1; u < 8; ++u) {
+            const size_t gv = gtc_of(u) * kDV + c4;
+            vr[u][0] = __ldg(reinterpret_cast<const uint2 *>(p.v + gv));
+            vr[u][1] = kBeta ? make_uint2(load_beta(u), 0u) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int t = tb + u;
             const bool in = live(u);
-            const uint2 vw_c[2] = {in ? vw_nx[0] : make_uint2(0, 0),
-                                   !in ? make_uint2(0, 0) : kBeta ? beta_val(vw_nx[1].x, u) : vw_nx[1]};
-            if (u + 1 < 8) {
-                const size_t gt = gtc_of(u + 1), gv = gt * kDV + c4;
-                vw_nx[0] = __ldg(reinterpret_cast<const uint2 *>(p.v + gv));
-                vw_nx[1] = kBeta ? make_uint2(load_beta(u + 1), 0u) : __ldg(reinterpret_cast<const uint2 *>(p.w + gv));
-            }
+            const uint2 vw_c[2] = {in ? vr[u][0] : make_uint2(0, 0),
+                                   !in ? make_uint2(0, 0) : kBeta ? beta_val(vr[u][1].x, u) : vr[u][1]};
             const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[0]);
             const __nv_bfloat162 *hw = reinterpret_cast<const __nv_bfloat162 *>(&vw_c[1]);
             float vh[4];
