@@ -337,6 +337,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kChainThreads, 1) gd
     tc::fence_before_sync();
     tc::cluster_sync();
     tc::fence_after_sync();
+    // launched as a programmatic dependent of the intra kernel: the set-up above
+    // may overlap that kernel's last CTAs; its records and flags are read only
+    // after this wait (a hardware wait for the whole prerequisite grid)
+    tc::grid_dependency_wait();
     const uint32_t tmem = *tslot;
     uint32_t phase = 0;
     uint32_t rph = 0u;                           // bit b: parity of record buffer b's next copy
@@ -1215,6 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int T = p.T, H = p.H;
     const int t0 = kC * win, wend = min(T, t0 + kC);
     uint8_t *rec = ws + (size_t)wi * kWinBytes;
+    tc::grid_launch_dependents();                 // the chain kernel may launch once every CTA has started
 
     float *lw = (float *)(sm + L::LW);
     float *yb = (float *)(sm + L::YB);
@@ -1756,9 +1761,9 @@ cudaError_t launch_fwd_tc(const FwdParams &fp, void *workspace, cudaStream_t str
     auto chain = fp.qk_raw ? gdn2_fwd_tc_kernel<true> : gdn2_fwd_tc_kernel<false>;
     e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    // clusters of two CTAs (value-column halves of one head), set by the kernel's attribute
-    chain<<<2 * fp.B * fp.H, kChainThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    // clusters of two CTAs (value-column halves of one head), set by the kernel's
+    // attribute; a programmatic dependent of the intra kernel
+    return tc::launch_dependent(chain, dim3(2 * fp.B * fp.H), dim3(kChainThreads), smem, stream, p);
 }
 
 }  // namespace gdelta

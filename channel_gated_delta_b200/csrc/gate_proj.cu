@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(proj_threads<kUp>(), 1)
     const uint32_t s_accf = s_empty + 8 * kPStages, s_acce = s_accf + 16, s_stall = s_acce + 16;
     uint32_t *tslot = (uint32_t *)(sm + L::MISC);
     volatile int *abort_flag = (volatile int *)(sm + L::MISC + 8);
+    if (!kUp) tc::grid_launch_dependents();       // the up launch may start once every down CTA has started
 
     if (tid == 0) {
         for (int s = 0; s < kPStages; ++s) {
@@ -186,6 +187,9 @@ __global__ void __launch_bounds__(proj_threads<kUp>(), 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    // the up launch is a programmatic dependent of the down launch: the codes are
+    // read only after this (hardware) wait for the whole down grid
+    if (kUp) tc::grid_dependency_wait();
     const uint32_t tmem = *tslot;
     bool timed_out = false;
 
@@ -522,8 +526,8 @@ cudaError_t launch_gate_proj(const GateProjParams &gp, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     p.nn = gp.d / kPN;
     p.jobs = mt * 5 * p.nn;
-    gate_proj_kernel<true><<<min(sms[dev], p.jobs), proj_threads<true>(), smem_up, stream>>>(ta, tb, om, p);
-    return cudaGetLastError();
+    return tc::launch_dependent(gate_proj_kernel<true>, dim3(min(sms[dev], p.jobs)), dim3(proj_threads<true>()),
+                                smem_up, stream, ta, tb, om, p);
 }
 
 }  // namespace gdelta

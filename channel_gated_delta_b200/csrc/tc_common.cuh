@@ -17,6 +17,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace gdelta {
 namespace tc {
 
@@ -206,6 +208,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- programmatic dependent launch ----
+// The next kernel in the stream, when launched with launch_dependent, may start
+// once every CTA of this grid has executed this (or exited).
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until the grid this one depends on has completed and its memory
+// operations are visible (returns at once when there is none).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- mbarriers (shared::cta) ----
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
@@ -389,6 +399,27 @@ __device__ __forceinline__ void ld_global_nc_v8(const void *p, uint4 &a, uint4 &
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Host: launch `kernel` as a programmatic dependent of the kernel before it in
+// `stream` (cudaLaunchAttributeProgrammaticStreamSerialization): its CTAs may
+// start once every CTA of that kernel has executed grid_launch_dependents, and
+// it must call grid_dependency_wait before reading what that kernel writes.
+// Cluster dimensions come from the kernel's own attribute.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace tc
