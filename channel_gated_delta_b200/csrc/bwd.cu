@@ -100,6 +100,12 @@ __device__ __forceinline__ void red_add(float *p, float x) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
 }
 
+// alpha = e^{log alpha} and 2 sigmoid(z) with the special-function unit's
+// exponential (relative error about 1e-6, far inside what the fp32 recurrence
+// needs); the exponent of the sigmoid is clamped so that its sum stays finite.
+__device__ __forceinline__ float alpha_of(float la) { return __expf(la); }
+__device__ __forceinline__ float two_sigmoid_bwd(float z) { return __fdividef(2.f, 1.f + __expf(fminf(-z, 80.f))); }
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 
@@ -229,12 +235,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     // the token's vectors into buffer bf (no barrier here: see TokBuf)
     auto stage = [&](const Tok &r, int ph, TokBuf &bf) {
         if (keyt) {
-            const float kk = cv(r.k0), al = expf(fl(r.k1));
+            const float kk = cv(r.k0), al = alpha_of(fl(r.k1));
             bf.k[tid] = kk;
             bf.kh[tid] = cv(r.k2) * kk;
             bf.al[tid] = al;
             if (ph == kF) bf.ka[tid] = kk * al;
-            if (ph != kRe) bf.qt[tid] = cv(r.k3) * gs_own * two_sigmoid(cv(r.k4));
+            if (ph != kRe) bf.qt[tid] = cv(r.k3) * gs_own * two_sigmoid_bwd(cv(r.k4));
         } else if (valt) {
             bf.vh[j] = cv(r.v0) * cv(r.v1);
             if (ph != kF) bf.r[j] = fl(r.v4);
@@ -515,7 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
                 const size_t gi = gt * kBD + tid;
                 const float kk = cb.k[tid], al = cb.al[tid];
                 const float bv = cv(cur.k2), qv = cv(cur.k3), zv = cv(cur.k4);
-                const float ts = two_sigmoid(zv);
+                const float ts = two_sigmoid_bwd(zv);
                 const float dqt = sm.rows[0][tid], dkh = sm.rows[2][tid];
                 red_add(p.grad_k + gi, sm.rows[1][tid] + al * sm.rows[3][tid] + bv * dkh);
                 red_add(p.grad_b + gi, kk * dkh);
