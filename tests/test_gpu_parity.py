@@ -629,6 +629,28 @@ def test_backward_long_sequence_matches_autograd_oracle():
     assert max(e.values()) <= TOL_BWD, e
 
 
+def test_backward_full_size_sampled_heads():
+    """The benchmark workload (B4 T4096 H16 bf16, the call `bench.py` times):
+    every token gradient of the first and the last head against the float64
+    autograd oracle (about 18 s of CPU a head); the other heads run in the
+    same launch."""
+    import channel_gated_delta_b200 as gd
+    from oracle import backward as ob
+    shape = synth.CONFIGS["muir1b3_bf16"]
+    inp = synth.generate(shape)
+    d = to_dev(inp)
+    dy = torch.randn(shape.B, shape.T, shape.H, 128, generator=torch.Generator().manual_seed(13))
+    g = gd.gdelta_bwd(d["q"], d["k"], d["v"], d["b"], d["w"], d["z"], d["g"], d["log_alpha"], dy.cuda(),
+                      gamma_stat=d["gamma_stat"])
+    torch.cuda.synchronize()
+    assert gd.gdelta_get_last_device_error() == 0
+    heads = [(0, 0), (shape.B - 1, shape.H - 1)]
+    ref = ob.backward(inp, dy.numpy(), heads=heads)
+    e = {key: err(sel_heads(g[key].cpu(), heads), ref["d" + key])
+         for key in ("q", "k", "v", "b", "w", "z", "g", "log_alpha")}
+    assert max(e.values()) <= TOL_BWD, e
+
+
 def test_backward_without_tokens_passes_the_state_gradient_through():
     import channel_gated_delta_b200 as gd
     B, H = 1, 2
