@@ -157,9 +157,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kBT, 1) gdn2_bwd_ker
     auto own_full = [&](int m) { return (size_t)row_of(m) * kBD + gc0 + col4; };  // in a [128][128] matrix
     // Two state tiles in shared memory (each a [128][64] half-matrix, the chunk
     // buffer's layout) and their mbarriers (a third one is never completed: the
-    // failure-path test waits on it).  The chunk's
-    // states move between them and the chunk buffer by bulk copies (one thread,
-    // 32 KiB each), which keeps that traffic off the threads' load/store path.
+    // failure-path test waits on it).  The chunk's states move between them and
+    // the chunk buffer by bulk copies (one thread, 32 KiB each), which keeps that
+    // traffic off the threads' load/store path.
     float *const slot0 = reinterpret_cast<float *>(dsm_base);
     auto slot = [&](int x) { return slot0 + (size_t)x * mat; };
     const uint32_t s_slot0 = tc::smem_u32(slot0), s_mb = s_slot0 + 2 * kSlotBytes;
