@@ -63,6 +63,7 @@ constexpr uint32_t kBwdDrainPolls = 1u << 22;    // polls of the wait that drain
 // The thread that issues the walk's state loads: in warp 6, which has no key or
 // value role, so that its proxy fence never waits on gradient atomics.
 constexpr int kLoader = 192;
+static_assert(kLoader >= kBD + kBH && kLoader < kBT, "the loader thread has no key or value role");
 
 // Reduce-scatter of 8 per-lane values over a half-warp: afterwards lane l
 // holds the sum over its 16 lanes of value (l >> 1) & 7.

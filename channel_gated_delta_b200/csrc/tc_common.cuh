@@ -17,8 +17,6 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include <utility>
-
 namespace gdelta {
 namespace tc {
 
@@ -405,7 +403,8 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 // `stream` (cudaLaunchAttributeProgrammaticStreamSerialization): its CTAs may
 // start once every CTA of that kernel has executed grid_launch_dependents, and
 // it must call grid_dependency_wait before reading what that kernel writes.
-// Cluster dimensions come from the kernel's own attribute.
+// Cluster dimensions come from the kernel's own attribute.  A runtime that
+// refuses the attribute gets an ordinary launch (then the wait returns at once).
 template <typename... Params, typename... Args>
 inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
                                     cudaStream_t stream, Args &&...args) {
@@ -419,7 +418,13 @@ inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 b
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) {
+        (void)cudaGetLastError();                 // clear the refusal, then launch in order
+        cfg.numAttrs = 0;
+        e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    }
+    return e;
 }
 
 }  // namespace tc
