@@ -116,10 +116,12 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms from before the
+    warm-up until after the last GPU measurement (the timed loops are too short
+    for the sampling period on their own; the GPU is under load throughout)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,utilization.gpu")
 
     def __init__(self, index: int):
         self.index = index
@@ -132,10 +134,16 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
-        time.sleep(0.3)
+            return
+        # wait (at most 5 s) until the first sample is written, so that sampling is live
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -148,7 +156,7 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
+            if len(parts) >= 10:
                 rows.append(parts)
         os.unlink(self.path)
         if not rows:
@@ -159,6 +167,11 @@ class ClockSampler:
                 return float(x)
             except ValueError:
                 return None
+        # samples taken while kernels ran (the window also holds host-only work,
+        # such as generating the other workloads' inputs); all of them if none
+        n_all = len(rows)
+        loaded = [r for r in rows if (num(r[9]) or 0.0) >= 50.0]
+        rows = loaded or rows
         sm = [num(r[1]) for r in rows if num(r[1]) is not None]
         mx = [num(r[2]) for r in rows if num(r[2]) is not None]
         pw = [num(r[3]) for r in rows if num(r[3]) is not None]
@@ -167,7 +180,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "power_w_max": max(pw) if pw else None,
-                "samples": len(rows), "reasons": reasons}
+                "samples": n_all, "samples_under_load": len(loaded), "reasons": reasons}
 
 
 def fwd_bytes(B, T, H, dk, dv, tok_bytes, z=True, beta=False, decay_tok=False):
@@ -253,14 +266,14 @@ def run_ours(args, rank, local, world):
         if ev is not None:
             ev[3].record(stream)
 
+    clocks = ClockSampler(dev.index if world == 1 else local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     if gd.gdelta_get_last_device_error(stream) != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    clocks = ClockSampler(dev.index if world == 1 else local)
-    clocks.start()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -271,7 +284,6 @@ def run_ours(args, rank, local, world):
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
-    clk = clocks.stop()
     total_ms = start.elapsed_time(end)
     fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms_step = max_over_ranks(total_ms / args.steps, world)
@@ -306,6 +318,9 @@ def run_ours(args, rank, local, world):
 
     # ---- end to end through the public API with host buffers
     e2e = None if args.no_e2e else run_e2e(args, gd, host, dev, stream, shape, world, path)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    clk["window"] = "from before the warm-up to the end of the last GPU measurement"
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -459,13 +474,13 @@ def run_forms(args, gd, d, shape, dev, stream, ws, world):
                                   S_in=S, S_out=S, y=y, chunk=C, path=args.path, workspace=ws,
                                   stream=stream, beta=beta, decay_per_token=f["decay_tok"], qk_raw=raw)
 
-        for _ in range(3):
+        for _ in range(5):
             gd.gdelta_state_init(S, stream=stream)
             call()
         torch.cuda.synchronize(dev)
         if gd.gdelta_get_last_device_error(stream) != 0:
             raise RuntimeError(f"device status word set during the {name} warm-up")
-        n = max(3, args.steps)
+        n = max(20, args.steps)                              # median of at least 20 calls
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         barrier(world)
         for i in range(n):
@@ -529,12 +544,12 @@ def run_configs(args, gd, dev, stream, rank, world):
                                   gamma_stat=d["gamma_stat"], S_in=None, S_out=S, y=y, chunk=C,
                                   path=args.path, workspace=ws, stream=stream)
 
-        for _ in range(3):
+        for _ in range(5):
             call()
         torch.cuda.synchronize(dev)
         if gd.gdelta_get_last_device_error(stream) != 0:
             raise RuntimeError(f"device status word set during the {name} warm-up")
-        n = max(3, min(args.steps, 10))
+        n = max(20, min(args.steps, 40))                     # median of at least 20 calls
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         barrier(world)
         for a, c in evs:
@@ -624,12 +639,12 @@ def run_gate_proj(args, gd, shape, dev, stream, rank, world):
         gd.gdelta_gate_proj(inp["x"], inp["w_down"], inp["w_up"], inp["bias"], ranks=ranks, out=out,
                             workspace=ws, stream=stream)
 
-    for _ in range(3):
+    for _ in range(5):
         call()
     torch.cuda.synchronize(dev)
     if gd.gdelta_get_last_device_error(stream) != 0:
         raise RuntimeError("device status word set during the gate projection warm-up")
-    n = max(3, min(args.steps, 20))
+    n = max(20, min(args.steps, 40))                         # median of at least 20 calls
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     barrier(world)
     for a, c in evs:
