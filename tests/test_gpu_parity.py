@@ -621,6 +621,15 @@ def test_backward_matches_autograd_oracle(B, T, H, dtype):
     assert max(e.values()) <= TOL_BWD, e
 
 
+@pytest.mark.parametrize("T", [33, 34, 35])
+def test_backward_short_last_chunk(T):
+    """A last checkpoint chunk of 1, 2 or 3 tokens: its states stay in the two
+    shared-memory tiles (1 and 2), one is bulk-loaded back from the checkpoint
+    (2), the first state goes through the chunk buffer (3)."""
+    e = bwd_errors(*_bwd_case(1, T, 2, "f32", 300 + T))
+    assert max(e.values()) <= TOL_BWD, e
+
+
 def test_backward_long_sequence_matches_autograd_oracle():
     """1024 tokens (32 checkpoint chunks) on every head of B2 H4 (the last
     batch row's last head included), bf16 tokens, a non-zero initial state and
